@@ -1,0 +1,139 @@
+"""Torch-tensor entry points over the C ABI: allocation of outputs and workspace
+(PyTorch's caching allocator) and argument marshalling; every step of the
+computation runs in libfa.so's CUDA kernels.  Inputs must be contiguous bf16
+CUDA tensors; anything else raises -- there is no CPU path.
+
+Shapes follow the flash-attention README (flash_attn_func, flash_attn_varlen_func,
+flash_attn_with_kvcache docstrings): q (B, Sq, Hq, D), k/v (B, Sk, Hkv, D); varlen
+q (total_q, Hq, D) with int32 cu_seqlens; caches (B, capacity, Hkv, D).
+softmax_scale defaults to 1/sqrt(D) (README, "How to use FlashAttention").
+"""
+
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import abi
+
+
+def _check(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _raise(status: int, where: str):
+    if status != abi.FA_OK:
+        raise abi.FAError(status, where)
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    # torch's allocator returns >= 512-byte aligned blocks
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def flash_attn_func(q, k, v, softmax_scale=None, causal=False):
+    """Forward: returns (out (B, Sq, Hq, D) bf16, lse (B, Hq, Sq) fp32)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
+    _raise(abi.fa_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal), "fa_fwd")
+    return out, lse
+
+
+def flash_attn_backward(dout, q, k, v, out, lse, softmax_scale=None, causal=False):
+    """Backward: returns (dq, dk, dv) shaped like q, k, v."""
+    for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check(t, n)
+    _check(lse, "lse", torch.float32)
+    B, Sq, Hq, D = q.shape
+    Sk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nb = abi.fa_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D)
+    ws = _workspace(nb, q.device)
+    _raise(abi.fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, scale, causal, ws, nb), "fa_bwd")
+    return dq, dk, dv
+
+
+def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale=None,
+                           causal=False):
+    """Packed forward: returns (out (total_q, Hq, D), lse (Hq, total_q))."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check(t, n)
+    _check(cu_seqlens_q, "cu_seqlens_q", torch.int32)
+    _check(cu_seqlens_k, "cu_seqlens_k", torch.int32)
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    nseq = cu_seqlens_q.numel() - 1
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
+    out = torch.empty_like(q)
+    lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    _raise(abi.fa_varlen_fwd(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q, max_seqlen_k,
+                             total_q, total_k, Hq, Hkv, D, scale, causal), "fa_varlen_fwd")
+    return out, lse
+
+
+def flash_attn_varlen_backward(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
+                               softmax_scale=None, causal=False):
+    for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")):
+        _check(t, n)
+    _check(lse, "lse", torch.float32)
+    total_q, Hq, D = q.shape
+    total_k, Hkv = k.shape[0], k.shape[1]
+    nseq = cu_seqlens_q.numel() - 1
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    nb = abi.fa_varlen_bwd_workspace_size(nseq, total_q, total_k, Hq, Hkv, D)
+    ws = _workspace(nb, q.device)
+    _raise(abi.fa_varlen_bwd(q, k, v, out, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q,
+                             max_seqlen_k, total_q, total_k, Hq, Hkv, D, scale, causal, ws, nb), "fa_varlen_bwd")
+    return dq, dk, dv
+
+
+def flash_attn_with_kvcache(q, k_cache, v_cache, cache_seqlens, softmax_scale=None, causal=False, num_splits=0,
+                            return_lse=True):
+    """Decode against a contiguous cache: returns (out (B, Sq, Hq, D), lse (B, Hq, Sq) or None)."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _check(t, n)
+    _check(cache_seqlens, "cache_seqlens", torch.int32)
+    B, Sq, Hq, D = q.shape
+    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device) if return_lse else None
+    nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, Sq, cap, D, num_splits)
+    ws = _workspace(nb, q.device)
+    _raise(abi.fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, out, lse, B, Hq, Hkv, Sq, cap, D, scale, causal,
+                              num_splits, ws, nb), "fa_fwd_kvcache")
+    return out, lse
+
+
+class FlashAttnFunction(torch.autograd.Function):
+    """Autograd wrapper: forward = fa_fwd, backward = fa_bwd."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, softmax_scale=None, causal=False):
+        out, lse = flash_attn_func(q, k, v, softmax_scale, causal)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.softmax_scale, ctx.causal = softmax_scale, causal
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = flash_attn_backward(dout.contiguous(), q, k, v, out, lse, ctx.softmax_scale, ctx.causal)
+        return dq, dk, dv, None, None

@@ -1,0 +1,606 @@
+// bwd.cu -- backward of exact tiled attention on sm_100a.
+//
+// The scores are recomputed from Q, K and the forward's LSE instead of being
+// stored (flash-attention README: IO-aware tiling with recomputation;
+// FlashAttention fork v1.4 notes, section 4: the backward applies the
+// exponential against the stored statistics, scale_apply_exp2 with
+// Scale_max = false).  With S = scale Q K^T, P = exp(S - LSE):
+//   dV = P^T dO,  dP = dO V^T,  Delta_i = rowsum(dO * O)_i,
+//   dS = P * (dP - Delta),  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three launches:
+//   1. preprocess: Delta = rowsum(dO * O) in fp32, LSE2 = LSE * log2(e) (+inf for
+//      rows with no key, so their P is exactly 0), and a zeroed fp32 dQ accumulator.
+//   2. main kernel, one persistent CTA per SM, KV-tile stationary: a work unit
+//      is (sequence, KV head, 128-key tile); it loops over the 128-row query
+//      tiles of every query head that reads the KV head (so dK and dV of GQA
+//      need no atomics) and, for causal masks, only over query tiles that can
+//      see the key tile.  Roles:
+//        warps 0-3  compute: thread = key row; P^T, dS^T from S^T and dP^T in
+//                   tensor memory; dK / dV epilogue
+//        warps 4-7  dQ: thread = query row; reads the dQ tile from tensor memory
+//                   and adds it to the fp32 accumulator (vector atomics)
+//        warp 8     producer: K, V once per unit; Q, dO tiles (TMA) and the
+//                   tile's LSE2 / Delta (plain loads) through a 2-stage ring
+//        warp 9     tensor memory and every tcgen05 MMA:
+//                   S^T = K Q^T, dP^T = V dO^T              (K-major x K-major)
+//                   dV += P^T dO, dK += dS^T Q               (tensor-memory A)
+//                   dQ = dS K                                (N-major x N-major)
+//   3. convert: dQ = bf16(scale * dQacc).
+#include "internal.h"
+#include "sm100.cuh"
+
+#include <math.h>
+
+namespace fa {
+
+struct BwdParams {
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* dq_acc;          // [Hq][D/4][Tq][4]
+    const float* lse2;      // [Hq][Tq]
+    const float* delta;     // [Hq][Tq]
+    const int32_t* cu_q;
+    const int32_t* cu_k;
+    int num_seqs, Sq, Sk, Tq, Tk, Hq, Hkv, group;
+    int n_blocks, num_units;
+    float scale, scale_log2;
+    int causal;
+    unsigned long long timeout_ns;
+    int* status;
+};
+
+struct BUnit {
+    int b, hk, q_start, k_start, Lq, Lk, n0, m_start, n_m, n_it;
+    bool skip;
+};
+
+__device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
+    BUnit t;
+    const int per_n = p.num_seqs * p.Hkv;
+    const int n = u / per_n;          // key tile; the first tiles have the most work under a causal mask
+    const int r = u % per_n;
+    t.b = r / p.Hkv;
+    t.hk = r % p.Hkv;
+    if (p.cu_q != nullptr) {
+        t.q_start = __ldg(p.cu_q + t.b);
+        t.Lq = __ldg(p.cu_q + t.b + 1) - t.q_start;
+        t.k_start = __ldg(p.cu_k + t.b);
+        t.Lk = __ldg(p.cu_k + t.b + 1) - t.k_start;
+        t.q_start = max(t.q_start, 0);
+        t.k_start = max(t.k_start, 0);
+        t.Lq = max(min(t.Lq, p.Tq - t.q_start), 0);
+        t.Lk = max(min(t.Lk, p.Tk - t.k_start), 0);
+    } else {
+        t.q_start = t.b * p.Sq;
+        t.Lq = p.Sq;
+        t.k_start = t.b * p.Sk;
+        t.Lk = p.Sk;
+    }
+    t.n0 = n * 128;
+    t.skip = t.n0 >= t.Lk;
+    int m_start = 0;
+    if (p.causal) {
+        const int first_row = t.n0 - (t.Lk - t.Lq);   // first query row that sees key n0
+        m_start = first_row > 0 ? first_row / 128 : 0;
+    }
+    const int m_end = (t.Lq + 127) / 128;
+    t.m_start = m_start;
+    t.n_m = m_end > m_start ? m_end - m_start : 0;
+    t.n_it = t.n_m * p.group;
+    return t;
+}
+
+template <int D>
+struct BwdCfg {
+    static constexpr int BM = 128, BN = 128, ST = 2;
+    static constexpr int NCHUNK = D / 64;
+    static constexpr uint32_t T_BYTES = 128 * D * 2;      // one 128-row tile of K, V, Q or dO
+    static constexpr uint32_t DS_BYTES = 128 * 128 * 2;   // dS^T [key][query]
+    // layout: K | V | Q[ST] | dO[ST] | dS | LSE2[ST][128] | Delta[ST][128] | barriers
+    static constexpr uint32_t OFF_K = 0, OFF_V = T_BYTES, OFF_Q = 2 * T_BYTES, OFF_DO = (2 + ST) * T_BYTES,
+                              OFF_DS = (2 + 2 * ST) * T_BYTES, OFF_STAT = OFF_DS + DS_BYTES,
+                              OFF_BAR = OFF_STAT + 2 * ST * 128 * 4;
+    static constexpr int NUM_BARS = 2 + 2 * ST + 5;
+    static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr uint32_t COL_DV = 0, COL_DK = D, COL_S = 2 * D, COL_DP = 2 * D + 128;
+    static_assert(2 * D + 256 <= 512, "tensor memory budget");
+};
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+               const __grid_constant__ BwdParams p) {
+    using C = BwdCfg<D>;
+    constexpr int ST = C::ST;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);          // [ST][128]
+    float* sDel = sLSE + ST * 128;                                       // [ST][128]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t b0 = smem_u32(bars);
+    const uint32_t kv_full = b0, kv_empty = b0 + 8;
+    auto q_full = [&](int s) { return b0 + 8u * (2 + s); };
+    auto q_empty = [&](int s) { return b0 + 8u * (2 + ST + s); };
+    const uint32_t s_full = b0 + 8u * (2 + 2 * ST), p_full = s_full + 8, dq_full = s_full + 16,
+                   dq_empty = s_full + 24, dkv_full = s_full + 32;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int PRODUCER = 8, MMA = 9;
+
+    if ((smem_u32(smem) & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0) atomicCAS(p.status, 0, 2);
+        return;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bars + 0, 1);
+        mbar_init(bars + 1, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(bars + 2 + s, 33);
+            mbar_init(bars + 2 + ST + s, 1);
+        }
+        mbar_init(bars + 2 + 2 * ST + 0, 1);    // s_full
+        mbar_init(bars + 2 + 2 * ST + 1, 128);  // p_full
+        mbar_init(bars + 2 + 2 * ST + 2, 1);    // dq_full
+        mbar_init(bars + 2 + 2 * ST + 3, 128);  // dq_empty
+        mbar_init(bars + 2 + 2 * ST + 4, 1);    // dkv_full
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == PRODUCER && lane == 0) {
+        tma_prefetch_map(&tmQ);
+        tma_prefetch_map(&tmK);
+        tma_prefetch_map(&tmV);
+        tma_prefetch_map(&tmDO);
+    }
+    if (warp == MMA) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Watch w{abort_flag, p.status, p.timeout_ns};
+    const int G = p.group;
+
+    if (warp == PRODUCER) {
+        // ------------------------------------------------------------ producer (whole warp)
+        uint32_t unit_it = 0, q_it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const BUnit t = decode_bunit(p, u);
+            if (t.skip || t.n_it == 0) continue;
+            if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(kv_full, 2 * C::T_BYTES);
+#pragma unroll
+                for (int c = 0; c < C::NCHUNK; ++c) {
+                    tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
+                                t.k_start + t.n0);
+                    tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
+                                t.k_start + t.n0);
+                }
+            }
+            ++unit_it;
+            for (int it = 0; it < t.n_it; ++it, ++q_it) {
+                const int g = it / t.n_m;
+                const int m0 = (t.m_start + it % t.n_m) * 128;
+                const int h = t.hk * G + g;
+                const int st = q_it % ST;
+                if (q_it >= ST && !mbar_wait(q_empty(st), ((q_it / ST) - 1) & 1, w)) { ok = false; break; }
+                // tile statistics; rows past the sequence get LSE2 = +inf (P = 0) and Delta = 0
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int qi = lane * 4 + e;
+                    const int row = m0 + qi;
+                    const bool in = row < t.Lq;
+                    const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
+                    sLSE[st * 128 + qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
+                    sDel[st * 128 + qi] = in ? __ldg(p.delta + idx) : 0.f;
+                }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(q_full(st), 2 * C::T_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c) {
+                        tma_load_3d(smem_u32(smem + C::OFF_Q + st * C::T_BYTES + c * 128 * 128), &tmQ, q_full(st),
+                                    c * 64, h, t.q_start + m0);
+                        tma_load_3d(smem_u32(smem + C::OFF_DO + st * C::T_BYTES + c * 128 * 128), &tmDO, q_full(st),
+                                    c * 64, h, t.q_start + m0);
+                    }
+                }
+                mbar_arrive(q_full(st));
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+            constexpr uint32_t id_tn = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
+            constexpr uint32_t id_mm = idesc_bf16_f32(128, D, true, true);       // dQ
+            uint32_t unit_it = 0, q_it = 0, g_it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const BUnit t = decode_bunit(p, u);
+                if (t.skip || t.n_it == 0) continue;
+                if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
+                for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
+                    const int st = q_it % ST;
+                    if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
+                    if (g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint8_t* sq = smem + C::OFF_Q + st * C::T_BYTES;
+                    const uint8_t* sdo = smem + C::OFF_DO + st * C::T_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+                        umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + o), 16, 1024),
+                                sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+                        umma_ss(tmem + C::COL_DP, sdesc_sw128(smem_u32(smem + C::OFF_V + o), 16, 1024),
+                                sdesc_sw128(smem_u32(sdo + o), 16, 1024), id_kk, kk > 0);
+                    }
+                    umma_commit(s_full);
+                    if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 query rows
+                        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                        umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8,
+                                sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                        umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8,
+                                sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
+                        umma_ss(tmem + C::COL_S,
+                                sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
+                                sdesc_sw128(smem_u32(smem + C::OFF_K + kk * 16 * 128), 128 * 128, 1024), id_mm,
+                                kk > 0);
+                    }
+                    umma_commit(dq_full);
+                    umma_commit(q_empty(st));
+                }
+                if (!ok) break;
+                umma_commit(dkv_full);
+                umma_commit(kv_empty);
+                ++unit_it;
+            }
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ------------------------------------------------------------ compute warpgroup (thread = key row)
+        const int r = warp * 32 + lane;
+        const uint32_t lb = tmem_lane_base(warp);
+        const float c2 = p.scale_log2;
+        uint32_t unit_it = 0, q_it = 0, g_it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const BUnit t = decode_bunit(p, u);
+            if (t.skip) continue;
+            const int kj = t.n0 + r;                 // key index inside the sequence
+            const bool kvalid = kj < t.Lk;
+            const size_t krow = (static_cast<size_t>(t.k_start) + kj) * p.Hkv + t.hk;
+            if (t.n_it == 0) {
+                if (kvalid) {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < D / 8; ++c) {
+                        reinterpret_cast<uint4*>(p.dk + krow * D)[c] = z;
+                        reinterpret_cast<uint4*>(p.dv + krow * D)[c] = z;
+                    }
+                }
+                continue;
+            }
+            const int off = t.Lk - t.Lq;
+            for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
+                const int m0 = (t.m_start + it % t.n_m) * 128;
+                const int st = q_it % ST;
+                if (!mbar_wait(s_full, g_it & 1, w)) { ok = false; break; }
+                if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
+                tc_fence_after();
+                // key kj may be seen by query row qi iff kj <= qi + off  <=>  qi >= kj - off
+                const int qmin = p.causal ? kj - off - m0 : -0x40000000;   // first allowed local query column
+                const bool full_row = kvalid && qmin <= 0;
+                const bool any_mask = __any_sync(0xffffffffu, !full_row);
+                const float* lse_t = sLSE + st * 128;
+                const float* del_t = sDel + st * 128;
+                uint8_t* ds_row = smem + C::OFF_DS + r * 128;
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t sa[32], da[32];
+                    tmem_ld32(tmem + lb + C::COL_S + cc * 32, sa);
+                    tmem_ld32(tmem + lb + C::COL_DP + cc * 32, da);
+                    tmem_ld_wait_tie(sa);
+                    reg_tie(da);
+                    uint32_t pp[16], dd[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4*>(lse_t + cc * 32 + e);
+                        const float4 d4 = *reinterpret_cast<const float4*>(del_t + cc * 32 + e);
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float pv[4], sv[4];
+#pragma unroll
+                        for (int x = 0; x < 4; ++x) {
+                            float pr = ex2_approx(fmaf(__uint_as_float(sa[e + x]), c2, -lv[x]));
+                            if (any_mask) {
+                                const int qc = cc * 32 + e + x;
+                                pr = (kvalid && qc >= qmin) ? pr : 0.f;
+                            }
+                            pv[x] = pr;
+                            sv[x] = pr * (__uint_as_float(da[e + x]) - dv[x]);
+                        }
+                        pp[e / 2] = pack_bf16x2(pv[0], pv[1]);
+                        pp[e / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
+                        dd[e / 2] = pack_bf16x2(sv[0], sv[1]);
+                        dd[e / 2 + 1] = pack_bf16x2(sv[2], sv[3]);
+                    }
+                    tmem_st16(tmem + lb + C::COL_S + cc * 16, pp);
+                    tmem_st16(tmem + lb + C::COL_DP + cc * 16, dd);
+                    // dS^T row r, query columns 32cc .. 32cc+31: 4 chunks of 16 bytes (128-byte swizzle)
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int chunk = cc * 4 + q4;               // 8 query columns per chunk
+                        const int box = chunk >> 3, cin = chunk & 7;
+                        *reinterpret_cast<uint4*>(ds_row + box * 128 * 128 + ((cin ^ (r & 7)) << 4)) =
+                            make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
+                    }
+                }
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (!ok) break;
+            // -------------------------------------------------- dK, dV epilogue
+            if (!mbar_wait(dkv_full, unit_it & 1, w)) { ok = false; break; }
+            ++unit_it;
+            tc_fence_after();
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = which == 0 ? C::COL_DV : C::COL_DK;
+                const float mul = which == 0 ? 1.f : p.scale;
+                __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + krow * D;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ra[32];
+                    tmem_ld32(tmem + lb + col + cc * 32, ra);
+                    tmem_ld_wait_tie(ra);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(ra[2 * e]) * mul, __uint_as_float(ra[2 * e + 1]) * mul);
+                    if (kvalid) {
+                        uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+        }
+    } else {
+        // ------------------------------------------------------------ dQ warpgroup (thread = query row)
+        const int wq = warp - 4;
+        const int r = wq * 32 + lane;
+        const uint32_t lb = tmem_lane_base(wq);
+        uint32_t g_it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const BUnit t = decode_bunit(p, u);
+            if (t.skip || t.n_it == 0) continue;
+            for (int it = 0; it < t.n_it; ++it, ++g_it) {
+                const int g = it / t.n_m;
+                const int m0 = (t.m_start + it % t.n_m) * 128;
+                const int h = t.hk * G + g;
+                const bool valid = m0 + r < t.Lq;
+                const size_t tok = static_cast<size_t>(t.q_start) + m0 + r;
+                if (!mbar_wait(dq_full, g_it & 1, w)) { ok = false; break; }
+                tc_fence_after();
+                float4* acc = reinterpret_cast<float4*>(p.dq_acc) + static_cast<size_t>(h) * (D / 4) * p.Tq + tok;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ra[32];
+                    tmem_ld32(tmem + lb + C::COL_S + cc * 32, ra);
+                    tmem_ld_wait_tie(ra);
+                    if (valid) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const float4 v = make_float4(__uint_as_float(ra[4 * e]), __uint_as_float(ra[4 * e + 1]),
+                                                         __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3]));
+                            atomicAdd(acc + static_cast<size_t>(cc * 8 + e) * p.Tq, v);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(dq_empty);
+            }
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) {
+        }
+    }
+    if (warp == MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ---------------------------------------------------------------------------- preprocess
+// One warp per (query token, head): Delta = sum_d dO * O (fp32), LSE2 = LSE * log2(e)
+// (+inf where LSE = -inf).  Also zeroes the dQ accumulator (grid-stride).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
+                                                      const float* lse, float* lse2, float* delta, float* dq_acc,
+                                                      int Tq, int Hq, int Sq, long long lse_sB, long long lse_sH,
+                                                      int lse_sT) {
+    const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    const long long rows = static_cast<long long>(Tq) * Hq;
+    {
+        const long long n4 = rows * D / 4;
+        float4* z = reinterpret_cast<float4*>(dq_acc);
+        for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+             i += static_cast<long long>(gridDim.x) * blockDim.x)
+            z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    for (long long row = gw; row < rows; row += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
+        const int tok = static_cast<int>(row / Hq), h = static_cast<int>(row % Hq);
+        constexpr int PER = D / 32;
+        const __nv_bfloat16* o = out + row * D + lane * PER;
+        const __nv_bfloat16* g = dout + row * D + lane * PER;
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < PER; e += 2) {
+            const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + e);
+            const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(g + e);
+            s = fmaf(__bfloat162float(a.x), __bfloat162float(b.x), s);
+            s = fmaf(__bfloat162float(a.y), __bfloat162float(b.y), s);
+        }
+#pragma unroll
+        for (int x = 16; x > 0; x >>= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
+        if (lane == 0) {
+            long long li;
+            if (lse_sT) {
+                li = h * lse_sH + tok;
+            } else {
+                const int b = tok / Sq, i = tok - b * Sq;
+                li = b * lse_sB + h * lse_sH + i;
+            }
+            const float l = lse[li];
+            const size_t wi = static_cast<size_t>(h) * Tq + tok;
+            lse2[wi] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+            delta[wi] = s;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------- convert
+// dQ[tok][h][:] = bf16(scale * dQacc[h][:/4][tok][:%4]); 32 tokens x D per block through shared memory.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_convert_kernel(const float* dq_acc, __nv_bfloat16* dq, int Tq, int Hq,
+                                                          float scale) {
+    __shared__ float tile[32][D + 4];
+    const int h = blockIdx.y;
+    const int t0 = blockIdx.x * 32;
+    for (int i = threadIdx.x; i < 32 * (D / 4); i += blockDim.x) {
+        const int d4 = i / 32, tt = i % 32;
+        if (t0 + tt < Tq) {
+            const float4 v =
+                reinterpret_cast<const float4*>(dq_acc)[(static_cast<size_t>(h) * (D / 4) + d4) * Tq + t0 + tt];
+            tile[tt][4 * d4 + 0] = v.x;
+            tile[tt][4 * d4 + 1] = v.y;
+            tile[tt][4 * d4 + 2] = v.z;
+            tile[tt][4 * d4 + 3] = v.w;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < 32 * (D / 2); i += blockDim.x) {
+        const int tt = i / (D / 2), d2 = i % (D / 2);
+        if (t0 + tt < Tq) {
+            const uint32_t v = pack_bf16x2(tile[tt][2 * d2] * scale, tile[tt][2 * d2 + 1] * scale);
+            reinterpret_cast<uint32_t*>(dq + (static_cast<size_t>(t0 + tt) * Hq + h) * D)[d2] = v;
+        }
+    }
+}
+
+size_t bwd_workspace_bytes(long long Tq, int Hq, int D) {
+    const size_t acc = static_cast<size_t>(Tq) * Hq * D * 4;
+    const size_t stat = static_cast<size_t>(Tq) * Hq * 4;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    return up(acc) + 2 * up(stat);
+}
+
+template <int D>
+static int run_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                   void* workspace, const Device& dev, cudaStream_t stream) {
+    using C = BwdCfg<D>;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    float* dq_acc = static_cast<float*>(workspace);
+    float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + up(static_cast<size_t>(pr.Tq) * pr.Hq * D * 4));
+    float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + up(static_cast<size_t>(pr.Tq) * pr.Hq * 4));
+
+    {
+        const long long rows = static_cast<long long>(pr.Tq) * pr.Hq;
+        long long blocks = (rows + 7) / 8;
+        const long long cap = static_cast<long long>(dev.num_sms) * 16;
+        if (blocks > cap) blocks = cap;
+        bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta, dq_acc,
+            pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+        if (cudaPeekAtLastError() != cudaSuccess) return 5;
+    }
+
+    alignas(64) CUtensorMap mq, mk, mv, mdo;
+    const uint64_t rq = static_cast<uint64_t>(pr.Hq) * D * 2, rk = static_cast<uint64_t>(pr.Hkv) * D * 2;
+    if (!make_map_3d_bf16(&mq, pr.q, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, 128)) return 5;
+    if (!make_map_3d_bf16(&mdo, dout, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, 128)) return 5;
+    if (!make_map_3d_bf16(&mk, pr.k, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+    if (!make_map_3d_bf16(&mv, pr.v, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+
+    BwdParams p;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.dq_acc = dq_acc;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.cu_q = pr.cu_q;
+    p.cu_k = pr.cu_k;
+    p.num_seqs = pr.num_seqs;
+    p.Sq = pr.Sq;
+    p.Sk = pr.Sk;
+    p.Tq = pr.Tq;
+    p.Tk = pr.Tk;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.group = pr.Hq / pr.Hkv;
+    p.n_blocks = (pr.Sk + 127) / 128;
+    const long long units = static_cast<long long>(p.n_blocks) * pr.num_seqs * pr.Hkv;
+    if (units > 0x7fffffffLL) return 2;
+    p.num_units = static_cast<int>(units);
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale * 1.4426950408889634f;
+    p.causal = pr.causal;
+    p.timeout_ns = dev.timeout_ns;
+    p.status = dev.status;
+
+    auto kern = bwd_kernel<D>;
+    static bool set[64] = {};
+    if (!set[dev.id & 63]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
+            cudaSuccess)
+            return 5;
+        set[dev.id & 63] = true;
+    }
+    const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
+    if (grid > 0) {
+        prof_before(1, stream);
+        kern<<<grid, 320, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        prof_after(1, stream);
+        if (cudaPeekAtLastError() != cudaSuccess) return 5;
+    }
+    dim3 cg((pr.Tq + 31) / 32, pr.Hq);
+    bwd_convert_kernel<D><<<cg, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), pr.Tq, pr.Hq, pr.scale);
+    return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
+}
+
+int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk, void* dv,
+               void* workspace, const Device& dev, cudaStream_t stream) {
+    switch (pr.D) {
+        case 64: return run_bwd<64>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
+        case 128: return run_bwd<128>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
+        default: return 2;
+    }
+}
+
+}  // namespace fa

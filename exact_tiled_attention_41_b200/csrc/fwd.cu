@@ -1,0 +1,495 @@
+// fwd.cu -- forward of exact tiled softmax attention on sm_100a.
+//
+// What it computes (flash-attention README, "How to use FlashAttention"):
+//   O = softmax(scale * Q K^T + mask) V,   LSE_i = ln sum_j exp(scale q_i.k_j)
+// tile by tile with an online softmax (FlashAttention fork v1.4 notes,
+// section 4, softmax_rescale_o / scale_apply_exp2: running row max and row sum,
+// exponentials taken as exp2 of one FMA with log2(e) folded into the scale, a
+// -inf row max replaced by 0), so the score matrix never leaves the SM.
+//
+// Design (one persistent CTA per SM):
+//   * warps 0..4*NQ-1: NQ softmax warpgroups; warpgroup i owns query tile i
+//     (128 rows) of the CTA's work unit, thread t owns row t: it reads its row
+//     of S from tensor memory, keeps the row max m and row sum l in registers,
+//     writes P (bf16) back into tensor memory, rescales its row of O when its
+//     reference max moves, and finally normalises and stores O and the LSE.
+//   * warp 4*NQ: TMA producer (Q tiles once per unit, K/V tiles through a
+//     KST-stage shared-memory ring, 128-byte swizzle).
+//   * warp 4*NQ+1: allocates tensor memory and issues every tcgen05 MMA:
+//     S_i = Q_i K^T (both operands K-major in shared memory) and
+//     O_i += P_i V (P from tensor memory, V N-major in shared memory).
+//   Order per KV tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the tensor
+//   core computes one tile's scores while the other tile's softmax runs.
+//   * work units (sequence, head, block of NQ*128 query rows) are taken
+//     round-robin in heaviest-first order (query blocks with most KV tiles first
+//     for causal masks); causal blocks stop at the last KV tile they can see.
+//
+// Exactness of the deferred rescale: P, l and O are all taken against the same
+// reference value m_ref of the row, which is only raised when a tile's max
+// exceeds it by more than kDeferLog2 (in log2 units).  softmax(x) is independent
+// of the reference subtracted, so the result is exact attention; the only effect
+// is that P may reach 2^kDeferLog2 before the final division (well inside
+// bf16/fp32 range).  With kDeferLog2 = 0 the reference follows every increase
+// of the running max.
+#include "internal.h"
+#include "sm100.cuh"
+
+#include <math.h>
+
+namespace fa {
+
+struct FwdParams {
+    __nv_bfloat16* o;
+    float* lse;
+    const int32_t* cu_q;
+    const int32_t* cu_k;
+    int num_seqs, Sq, Sk, Tq, Tk, Hq, Hkv, group;
+    int m_blocks, num_units;
+    float scale_log2;
+    int causal;
+    long long lse_sB, lse_sH;
+    int lse_sT;
+    unsigned long long timeout_ns;
+    int* status;
+};
+
+struct Unit {
+    int b, h, q_start, k_start, Lq, Lk, q0, n_kv;
+    bool skip;
+};
+
+template <int ROWS, int BK>
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+    Unit t;
+    const int per_m = p.num_seqs * p.Hq;
+    const int m = p.m_blocks - 1 - u / per_m;
+    const int r = u % per_m;
+    t.b = r / p.Hq;
+    t.h = r % p.Hq;
+    if (p.cu_q != nullptr) {
+        t.q_start = __ldg(p.cu_q + t.b);
+        t.Lq = __ldg(p.cu_q + t.b + 1) - t.q_start;
+        t.k_start = __ldg(p.cu_k + t.b);
+        t.Lk = __ldg(p.cu_k + t.b + 1) - t.k_start;
+        // malformed offsets can only shrink the work: rows are clipped to the tensors
+        t.q_start = max(t.q_start, 0);
+        t.k_start = max(t.k_start, 0);
+        t.Lq = max(min(t.Lq, p.Tq - t.q_start), 0);
+        t.Lk = max(min(t.Lk, p.Tk - t.k_start), 0);
+    } else {
+        t.q_start = t.b * p.Sq;
+        t.Lq = p.Sq;
+        t.k_start = t.b * p.Sk;
+        t.Lk = p.Sk;
+    }
+    t.q0 = m * ROWS;
+    t.skip = t.q0 >= t.Lq;
+    int kend = t.Lk;
+    if (p.causal) {
+        const int last_row = min(t.q0 + ROWS, t.Lq) - 1;
+        kend = min(kend, last_row + (t.Lk - t.Lq) + 1);
+    }
+    t.n_kv = kend > 0 ? (kend + BK - 1) / BK : 0;
+    return t;
+}
+
+template <int D, int NQ, int BK, int KST>
+struct FwdCfg {
+    static constexpr int BM = 128;
+    static constexpr int NCHUNK = D / 64;
+    static constexpr uint32_t Q_BYTES = BM * D * 2;
+    static constexpr uint32_t KV_BYTES = BK * D * 2;
+    static constexpr int NUM_BARS = 5 * NQ + 4 * KST;
+    static constexpr size_t SMEM = 1024 + NQ * Q_BYTES + 2 * KST * KV_BYTES + NUM_BARS * 8 + 16;
+    static constexpr int THREADS = (4 * NQ + 2) * 32;
+    static constexpr uint32_t S_COL(int i) { return i * BK; }
+    static constexpr uint32_t O_COL(int i) { return NQ * BK + i * D; }
+    static_assert(NQ * BK + NQ * D <= 512, "tensor memory budget");
+    static_assert(D % 64 == 0 && BK % 64 == 0, "tile shape");
+};
+
+constexpr float kDeferLog2 = 8.0f;
+constexpr float kLn2 = 0.69314718055994530942f;
+
+template <int D, int NQ, int BK, int KST>
+__global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
+    using C = FwdCfg<D, NQ, BK, KST>;
+    constexpr int BM = C::BM;
+    constexpr int ROWS = BM * NQ;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + NQ * C::Q_BYTES;
+    uint8_t* sV = sK + KST * C::KV_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + KST * C::KV_BYTES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const uint32_t bar0 = smem_u32(bars);
+    auto q_full = [&](int i) { return bar0 + 8u * (0 * NQ + i); };
+    auto q_empty = [&](int i) { return bar0 + 8u * (1 * NQ + i); };
+    auto s_full = [&](int i) { return bar0 + 8u * (2 * NQ + i); };
+    auto p_full = [&](int i) { return bar0 + 8u * (3 * NQ + i); };
+    auto o_full = [&](int i) { return bar0 + 8u * (4 * NQ + i); };
+    auto k_full = [&](int s) { return bar0 + 8u * (5 * NQ + s); };
+    auto k_empty = [&](int s) { return bar0 + 8u * (5 * NQ + KST + s); };
+    auto v_full = [&](int s) { return bar0 + 8u * (5 * NQ + 2 * KST + s); };
+    auto v_empty = [&](int s) { return bar0 + 8u * (5 * NQ + 3 * KST + s); };
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    constexpr int PRODUCER = 4 * NQ;
+    constexpr int MMA = 4 * NQ + 1;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NQ; ++i) {
+            mbar_init(bars + 0 * NQ + i, 1);
+            mbar_init(bars + 1 * NQ + i, 1);
+            mbar_init(bars + 2 * NQ + i, 1);
+            mbar_init(bars + 3 * NQ + i, 128);
+            mbar_init(bars + 4 * NQ + i, 1);
+        }
+        for (int s = 0; s < 4 * KST; ++s) mbar_init(bars + 5 * NQ + s, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == PRODUCER && lane == 0) {
+        tma_prefetch_map(&tmQ);
+        tma_prefetch_map(&tmK);
+        tma_prefetch_map(&tmV);
+    }
+    if (warp == MMA) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Watch w{abort_flag, p.status, p.timeout_ns};
+
+    if (warp == PRODUCER) {
+        if (lane == 0) {
+            uint32_t kv_it = 0, q_it = 0;
+            for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+                const Unit t = decode_unit<ROWS, BK>(p, u);
+                if (t.skip || t.n_kv == 0) continue;
+                const int hk = t.h / p.group;
+                bool ok = true;
+                for (int i = 0; i < NQ && ok; ++i) {
+                    if (q_it > 0 && !mbar_wait(q_empty(i), (q_it - 1) & 1, w)) ok = false;
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(q_full(i), C::Q_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_3d(smem_u32(sQ + i * C::Q_BYTES + c * BM * 128), &tmQ, q_full(i), c * 64, t.h,
+                                    t.q_start + t.q0 + i * BM);
+                }
+                if (!ok) break;
+                ++q_it;
+                for (int j = 0; j < t.n_kv && ok; ++j, ++kv_it) {
+                    const int st = kv_it % KST;
+                    const uint32_t n = kv_it / KST;
+                    if (n > 0 && !mbar_wait(k_empty(st), (n - 1) & 1, w)) { ok = false; break; }
+                    mbar_arrive_expect_tx(k_full(st), C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_3d(smem_u32(sK + st * C::KV_BYTES + c * BK * 128), &tmK, k_full(st), c * 64, hk,
+                                    t.k_start + j * BK);
+                    if (n > 0 && !mbar_wait(v_empty(st), (n - 1) & 1, w)) { ok = false; break; }
+                    mbar_arrive_expect_tx(v_full(st), C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_3d(smem_u32(sV + st * C::KV_BYTES + c * BK * 128), &tmV, v_full(st), c * 64, hk,
+                                    t.k_start + j * BK);
+                }
+                if (!ok) break;
+            }
+        }
+        __syncwarp();
+    } else if (warp == MMA) {
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BK, false, false);
+            constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
+            auto issue_qk = [&](int i, int st) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t qa = smem_u32(sQ + i * C::Q_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32);
+                    const uint32_t kb = smem_u32(sK + st * C::KV_BYTES + (kk >> 2) * BK * 128 + (kk & 3) * 32);
+                    umma_ss(tmem + C::S_COL(i), sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), idesc_qk,
+                            kk > 0 ? 1u : 0u);
+                }
+            };
+            auto issue_pv = [&](int i, int st, bool acc) {
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t vb = smem_u32(sV + st * C::KV_BYTES + kk * 16 * 128);
+                    umma_ts(tmem + C::O_COL(i), tmem + C::S_COL(i) + kk * 8, sdesc_sw128(vb, BK * 128, 1024),
+                            idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            uint32_t kv_it = 0, q_it = 0, p_it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const Unit t = decode_unit<ROWS, BK>(p, u);
+                if (t.skip || t.n_kv == 0) continue;
+                for (int i = 0; i < NQ && ok; ++i)
+                    if (!mbar_wait(q_full(i), q_it & 1, w)) ok = false;
+                if (!ok) break;
+                ++q_it;
+                {
+                    const int st = kv_it % KST;
+                    if (!mbar_wait(k_full(st), (kv_it / KST) & 1, w)) break;
+                    tc_fence_after();
+                    for (int i = 0; i < NQ; ++i) {
+                        issue_qk(i, st);
+                        umma_commit(s_full(i));
+                    }
+                    umma_commit(k_empty(st));
+                    if (t.n_kv == 1)
+                        for (int i = 0; i < NQ; ++i) umma_commit(q_empty(i));
+                }
+                for (int j = 0; j < t.n_kv && ok; ++j) {
+                    const uint32_t cur = kv_it + j;
+                    const int st = cur % KST;
+                    const uint32_t nxt = cur + 1;
+                    const int stn = nxt % KST;
+                    const bool has_next = j + 1 < t.n_kv;
+                    if (!mbar_wait(v_full(st), (cur / KST) & 1, w)) { ok = false; break; }
+                    tc_fence_after();
+                    for (int i = 0; i < NQ; ++i) {
+                        if (!mbar_wait(p_full(i), p_it & 1, w)) { ok = false; break; }
+                        tc_fence_after();
+                        issue_pv(i, st, j > 0);
+                        umma_commit(o_full(i));
+                        if (has_next) {
+                            if (i == 0) {
+                                if (!mbar_wait(k_full(stn), (nxt / KST) & 1, w)) { ok = false; break; }
+                                tc_fence_after();
+                            }
+                            issue_qk(i, stn);
+                            umma_commit(s_full(i));
+                        }
+                    }
+                    if (!ok) break;
+                    ++p_it;
+                    umma_commit(v_empty(st));
+                    if (has_next) {
+                        umma_commit(k_empty(stn));
+                        if (j + 2 == t.n_kv)
+                            for (int i = 0; i < NQ; ++i) umma_commit(q_empty(i));
+                    }
+                }
+                kv_it += t.n_kv;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------- softmax warpgroups
+        const int i = warp >> 2;
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;
+        const uint32_t lane_base = tmem_lane_base(wq);
+        const uint32_t tS = tmem + lane_base + C::S_COL(i);
+        const uint32_t tO = tmem + lane_base + C::O_COL(i);
+        const float c2 = p.scale_log2;
+        uint32_t s_it = 0, pv_total = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const Unit t = decode_unit<ROWS, BK>(p, u);
+            if (t.skip) continue;
+            const int row = t.q0 + i * BM + r;
+            const bool valid = row < t.Lq;
+            __nv_bfloat16* orow = p.o + (static_cast<size_t>(t.q_start + row) * p.Hq + t.h) * D;
+            float* lse_ptr = p.lse + t.b * p.lse_sB + t.h * p.lse_sH + static_cast<long long>(t.q_start) * p.lse_sT + row;
+            if (t.n_kv == 0) {
+                if (valid) {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
+                    *lse_ptr = -INFINITY;
+                }
+                continue;
+            }
+            const int off = t.Lk - t.Lq;
+            const int key_lim = p.causal ? min(t.Lk - 1, row + off) : (t.Lk - 1);
+            float m_ref = -INFINITY;
+            float l = 0.f;
+            for (int j = 0; j < t.n_kv; ++j) {
+                if (!mbar_wait(s_full(i), s_it & 1, w)) { ok = false; break; }
+                ++s_it;
+                tc_fence_after();
+                float s[BK];
+                {
+                    uint32_t ra[32];
+#pragma unroll
+                    for (int cc = 0; cc < BK / 32; ++cc) {
+                        tmem_ld32(tS + cc * 32, ra);
+                        tmem_ld_wait_tie(ra);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(ra[e]);
+                    }
+                }
+                const int kbase = j * BK;
+                if (__any_sync(0xffffffffu, kbase + BK - 1 > key_lim)) {
+#pragma unroll
+                    for (int c = 0; c < BK; ++c) s[c] = (kbase + c <= key_lim) ? s[c] : -INFINITY;
+                }
+                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+                for (int c = 4; c < BK; c += 4) {
+                    mx0 = fmaxf(mx0, s[c]);
+                    mx1 = fmaxf(mx1, s[c + 1]);
+                    mx2 = fmaxf(mx2, s[c + 2]);
+                    mx3 = fmaxf(mx3, s[c + 3]);
+                }
+                const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                const bool need = (mt - m_ref) * c2 > kDeferLog2;   // NaN (both -inf) -> false
+                if (__any_sync(0xffffffffu, need)) {
+                    const float m_new = fmaxf(m_ref, mt);
+                    const float alpha = (m_ref == -INFINITY) ? 0.f : ex2_approx((m_ref - m_new) * c2);
+                    const bool rescale = (j > 0) && __any_sync(0xffffffffu, m_ref != -INFINITY && alpha < 1.f);
+                    if (rescale) {
+                        if (!mbar_wait(o_full(i), (pv_total + j - 1) & 1, w)) { ok = false; }
+                        // all lanes reach here together; the abort case skips the work
+                        if (__all_sync(0xffffffffu, ok)) {
+                            tc_fence_after();
+                            uint32_t ro[32];
+#pragma unroll 1
+                            for (int cc = 0; cc < D / 32; ++cc) {
+                                tmem_ld32(tO + cc * 32, ro);
+                                tmem_ld_wait_tie(ro);
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+                                tmem_st32(tO + cc * 32, ro);
+                            }
+                            tmem_st_wait();
+                        } else {
+                            ok = false;
+                            break;
+                        }
+                    }
+                    l *= alpha;
+                    m_ref = m_new;
+                }
+                const float ms = (m_ref == -INFINITY) ? 0.f : m_ref * c2;
+                float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+                for (int half = 0; half < BK / 64; ++half) {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float a = ex2_approx(fmaf(s[half * 64 + 2 * e], c2, -ms));
+                        const float b = ex2_approx(fmaf(s[half * 64 + 2 * e + 1], c2, -ms));
+                        sum0 += a;
+                        sum1 += b;
+                        pk[e] = pack_bf16x2(a, b);
+                    }
+                    tmem_st32(tS + half * 32, pk);
+                }
+                l += sum0 + sum1;
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(p_full(i));
+            }
+            if (!ok) break;
+            pv_total += t.n_kv;
+            // ------------------------------------------------ epilogue: O / l, LSE
+            if (!mbar_wait(o_full(i), (pv_total - 1) & 1, w)) { ok = false; break; }
+            tc_fence_after();
+            const float inv_l = l > 0.f ? 1.f / l : 0.f;
+            uint32_t ro[32];
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                tmem_ld32(tO + cc * 32, ro);
+                tmem_ld_wait_tie(ro);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    pk[e] = pack_bf16x2(__uint_as_float(ro[2 * e]) * inv_l, __uint_as_float(ro[2 * e + 1]) * inv_l);
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+            if (valid) *lse_ptr = l > 0.f ? (m_ref * c2 + log2f(l)) * kLn2 : -INFINITY;
+            tc_fence_before();
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
+        // give tensor-core and TMA work already issued time to land before freeing
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) {
+        }
+    }
+    if (warp == MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int D, int NQ, int BK, int KST>
+static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream) {
+    using C = FwdCfg<D, NQ, BK, KST>;
+    alignas(64) CUtensorMap mq, mk, mv;
+    const uint64_t rq = static_cast<uint64_t>(pr.Hq) * D * 2, rk = static_cast<uint64_t>(pr.Hkv) * D * 2;
+    if (!make_map_3d_bf16(&mq, pr.q, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, C::BM)) return 5;
+    if (!make_map_3d_bf16(&mk, pr.k, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, BK)) return 5;
+    if (!make_map_3d_bf16(&mv, pr.v, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, BK)) return 5;
+
+    FwdParams p;
+    p.o = static_cast<__nv_bfloat16*>(out);
+    p.lse = lse;
+    p.cu_q = pr.cu_q;
+    p.cu_k = pr.cu_k;
+    p.num_seqs = pr.num_seqs;
+    p.Sq = pr.Sq;
+    p.Sk = pr.Sk;
+    p.Tq = pr.Tq;
+    p.Tk = pr.Tk;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.group = pr.Hq / pr.Hkv;
+    p.m_blocks = (pr.Sq + C::BM * NQ - 1) / (C::BM * NQ);
+    const long long units = static_cast<long long>(p.m_blocks) * pr.num_seqs * pr.Hq;
+    if (units > 0x7fffffffLL) return 2;
+    p.num_units = static_cast<int>(units);
+    p.scale_log2 = pr.scale * 1.4426950408889634f;
+    p.causal = pr.causal;
+    p.lse_sB = pr.lse_sB;
+    p.lse_sH = pr.lse_sH;
+    p.lse_sT = pr.lse_sT;
+    p.timeout_ns = dev.timeout_ns;
+    p.status = dev.status;
+    if (p.num_units == 0) return 0;
+
+    auto kern = fwd_kernel<D, NQ, BK, KST>;
+    static bool attr_set[64] = {};
+    if (!attr_set[dev.id & 63]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
+            cudaSuccess)
+            return 5;
+        attr_set[dev.id & 63] = true;
+    }
+    const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
+    prof_before(0, stream);
+    kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, p);
+    prof_after(0, stream);
+    return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
+}
+
+int launch_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream) {
+    switch (pr.D) {
+        case 64: return run_fwd<64, 2, 128, 4>(pr, out, lse, dev, stream);
+        case 128: return run_fwd<128, 2, 128, 2>(pr, out, lse, dev, stream);
+        case 256: return run_fwd<256, 1, 128, 1>(pr, out, lse, dev, stream);
+        default: return 2;
+    }
+}
+
+}  // namespace fa

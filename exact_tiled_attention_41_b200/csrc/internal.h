@@ -1,0 +1,78 @@
+// internal.h -- launch descriptors shared by the C-ABI layer (api.cu) and the
+// kernel files.  Host-side only types; no torch, no STL containers.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fa {
+
+// A batch of independent attention problems.  Dense batches are the special
+// case cu_q = cu_k = NULL with sequence b occupying tokens b*Sq .. b*Sq+Sq-1
+// (queries) and b*Sk .. b*Sk+Sk-1 (keys).
+struct Problem {
+    const void* q;       // [Tq, Hq, D]  bf16
+    const void* k;       // [Tk, Hkv, D] bf16
+    const void* v;       // [Tk, Hkv, D] bf16
+    const int32_t* cu_q; // device [num_seqs + 1] or NULL
+    const int32_t* cu_k;
+    int num_seqs;
+    int Sq, Sk;          // dense lengths, or the maxima for varlen
+    int Tq, Tk;          // total tokens
+    int Hq, Hkv, D;
+    float scale;
+    int causal;
+    // LSE addressing: index = b * lse_sB + h * lse_sH + tok_start * lse_sT + row
+    long long lse_sB, lse_sH;
+    int lse_sT;
+};
+
+struct Device {
+    int id;
+    int num_sms;
+    int* status;                 // device status word
+    unsigned long long timeout_ns;
+};
+
+int get_device(Device* dev);     // fills for the current device; returns FA status
+
+// optional CUDA-event timing around a main-kernel launch (see fa_profile_begin)
+void prof_before(int kernel_id, cudaStream_t s);
+void prof_after(int kernel_id, cudaStream_t s);
+
+int launch_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream);
+
+size_t bwd_workspace_bytes(long long Tq, int Hq, int D);
+int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
+               void* dv, void* workspace, const Device& dev, cudaStream_t stream);
+
+struct Decode {
+    const void* q;            // [B, 1, Hq, D]
+    const void* k_cache;      // [B, cap, Hkv, D]
+    const void* v_cache;
+    const int32_t* seqlens;   // device [B]
+    void* out;                // [B, 1, Hq, D]
+    float* lse;               // [B, Hq, 1] or NULL
+    int B, Hq, Hkv, cap, D;
+    float scale;
+    int chunk;                // keys per split (multiple of 64)
+    int max_chunks;           // ceil(cap / chunk)
+    float* part_o;            // [B, Hkv, max_chunks, group, D]
+    float* part_lse;          // [B, Hkv, max_chunks, group]
+};
+
+int decode_chunk_size(int B, int Hkv, int cap, int num_splits, int num_sms);
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int cap, int D, int chunk);
+int launch_decode(const Decode& d, const Device& dev, cudaStream_t stream);
+
+int launch_wait_selftest(unsigned long long timeout_ns, const Device& dev, cudaStream_t stream);
+int launch_umma_selftest(const void* a, const void* b, float* c, int mode, const Device& dev, cudaStream_t stream);
+
+// cuTensorMapEncodeTiled, fetched through the runtime so the library needs no -lcuda.
+bool make_map_3d_bf16(void* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1_bytes,
+                      uint64_t stride2_bytes, uint32_t box0, uint32_t box1, uint32_t box2);
+bool make_map_2d_bf16(void* map, const void* base, uint64_t d0, uint64_t d1, uint64_t stride1_bytes, uint32_t box0,
+                      uint32_t box1);
+
+}  // namespace fa

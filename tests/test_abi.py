@@ -1,0 +1,123 @@
+"""CPU checks of the C-ABI boundary: the library loads, exports every symbol the
+header declares, and rejects bad arguments before touching the GPU."""
+
+import os
+import re
+
+import pytest
+
+from exact_tiled_attention_41_b200 import abi
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "fa.h")
+FAKE = 0x10000        # a 16-byte aligned address that is never dereferenced (validation fails first)
+S0 = 0                # default stream handle
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(abi.LIB_PATH):
+        from exact_tiled_attention_41_b200 import build
+        build.build()
+    return abi.load()
+
+
+def test_header_declares_the_five_entry_points():
+    syms = declared_symbols()
+    for name in ("fa_fwd", "fa_bwd", "fa_varlen_fwd", "fa_varlen_bwd", "fa_fwd_kvcache"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(lib):
+    syms = declared_symbols()
+    assert len(syms) >= 15
+    for name in syms:
+        assert hasattr(lib, name), name
+    assert set(syms) == set(abi.EXPORTS)
+
+
+def test_status_strings(lib):
+    assert abi.status_string(0) == "ok"
+    assert "timed out" in abi.status_string(abi.FA_ERR_TIMEOUT)
+    assert abi.status_string(99) == "unknown status"
+
+
+def _fwd(**kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, B=1, Hq=4, Hkv=2, Sq=128, Sk=128, D=128,
+             softmax_scale=0.1, causal=1, stream=S0)
+    a.update(kw)
+    return abi.fa_fwd(**a)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(q=None), abi.FA_ERR_INVALID_ARG),
+    (dict(out=None), abi.FA_ERR_INVALID_ARG),
+    (dict(lse=None), abi.FA_ERR_INVALID_ARG),
+    (dict(B=0), abi.FA_ERR_INVALID_ARG),
+    (dict(Sq=0), abi.FA_ERR_INVALID_ARG),
+    (dict(Sk=-1), abi.FA_ERR_INVALID_ARG),
+    (dict(Hq=3, Hkv=2), abi.FA_ERR_INVALID_ARG),        # README: Hq must be divisible by Hkv
+    (dict(softmax_scale=0.0), abi.FA_ERR_INVALID_ARG),
+    (dict(softmax_scale=float("nan")), abi.FA_ERR_INVALID_ARG),
+    (dict(D=96), abi.FA_ERR_UNSUPPORTED),
+    (dict(D=512), abi.FA_ERR_UNSUPPORTED),                # README: head dims up to 256
+    (dict(q=FAKE + 8), abi.FA_ERR_ALIGNMENT),
+    (dict(out=FAKE + 2), abi.FA_ERR_ALIGNMENT),
+])
+def test_fwd_rejects_bad_arguments(lib, kw, want):
+    assert _fwd(**kw) == want
+
+
+def test_bwd_checks_workspace_before_launch(lib):
+    need = abi.fa_bwd_workspace_size(2, 4, 2, 300, 300, 128)
+    assert need >= 2 * 300 * 4 * 128 * 4       # fp32 dq accumulator at least
+    st = abi.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 300, 300, 128, 0.1, 1,
+                    FAKE, need - 1, S0)
+    assert st == abi.FA_ERR_WORKSPACE
+    st = abi.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 300, 300, 128, 0.1, 1,
+                    FAKE + 16, need, S0)
+    assert st == abi.FA_ERR_ALIGNMENT          # workspace must be 256-byte aligned
+    st = abi.fa_bwd(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 300, 300, 128, 0.1, 1,
+                    FAKE, need, S0)
+    assert st == abi.FA_ERR_INVALID_ARG
+
+
+def test_varlen_rejects_missing_cu_seqlens(lib):
+    st = abi.fa_varlen_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 2, 10, 10, 20, 20, 2, 2, 64, 0.1, 1, stream=S0)
+    assert st == abi.FA_ERR_INVALID_ARG
+    st = abi.fa_varlen_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, 2, 10, 10, 20, 20, 2, 2, 64, 0.1, 1, stream=S0)
+    assert st == abi.FA_ERR_ALIGNMENT
+    assert abi.fa_varlen_fwd_workspace_size(2, 20, 20, 2, 2, 64) == 0
+    assert abi.fa_varlen_bwd_workspace_size(2, 20, 20, 2, 2, 64) > 0
+
+
+def test_kvcache_argument_rules(lib):
+    need = abi.fa_fwd_kvcache_workspace_size(64, 32, 8, 1, 16384, 128, 0)
+    assert need > 0
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, None, 64, 32, 8, 1, 16384, 128, 0.1, 0, 0, FAKE, need, S0]
+    bad_sq = list(args)
+    bad_sq[9] = 2                                 # one query per row in this version
+    assert abi.fa_fwd_kvcache(*bad_sq) == abi.FA_ERR_INVALID_ARG
+    small = list(args)
+    small[16] = need - 1
+    assert abi.fa_fwd_kvcache(*small) == abi.FA_ERR_WORKSPACE
+    no_seqlens = list(args)
+    no_seqlens[3] = None
+    assert abi.fa_fwd_kvcache(*no_seqlens) == abi.FA_ERR_INVALID_ARG
+    # more splits need more partial storage
+    assert abi.fa_fwd_kvcache_workspace_size(64, 32, 8, 1, 16384, 128, 64) > abi.fa_fwd_kvcache_workspace_size(
+        64, 32, 8, 1, 16384, 128, 4)
+
+
+def test_product_path_has_no_oracle_or_cpu_fallback():
+    pkg = os.path.join(ROOT, "exact_tiled_attention_41_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in text and "from oracle" not in text, f
