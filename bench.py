@@ -1,0 +1,463 @@
+#!/usr/bin/env python
+"""Benchmark of exact tiled attention on B200.
+
+One step = forward + backward (O, LSE, dQ, dK, dV) of the dense causal
+prefill workload B=4, H=16, S=2048, D=128 (bf16, i.i.d. N(0,1) synthetic
+inputs), i.e. every row of the hot path: tile staging, QK^T, masking, online
+softmax, exact rescale, PV, epilogue, backward preprocess, backward main,
+dQ convert, on the persistent LPT schedule.  The metric is algorithmic
+TFLOP/s: forward 4*B*H*S^2*D/2 (causal), backward 2.5x that.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+N > 1 runs N independent replicas (one process per GPU, launched with
+torch.distributed.run); the work does not shard, so scaling is weak and the
+value is the sum over ranks of the work divided by the slowest rank's time.
+Rank 0 prints one JSON line.  ``--impl reference`` times the fp64 CPU oracle on
+a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd & bwd TFLOP/s (bf16, causal, D=128) and % of B200 dense BF16 peak"
+WORKLOAD = dict(workload="dense_prefill_B4_H16_S2048_D128_causal_fwd+bwd", batch_per_gpu=4, heads=16,
+                seq_len=2048, head_dim=128, causal=True)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def fwd_flops(B, H, Sq, Sk, D, causal):
+    return 4.0 * B * H * Sq * Sk * D * (0.5 if causal else 1.0)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return FALLBACK_PEAKS, "fallback"
+
+
+def traffic_record(kernel_name, source_file):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "roofline_traffic.txt")
+    try:
+        sha = hashlib.sha256(open(os.path.join(ROOT, source_file), "rb").read()).hexdigest()[:16]
+        for line in open(path):
+            f = dict(kv.split("=", 1) for kv in line.split() if "=" in kv)
+            if f.get("kernel") == kernel_name and f.get("source_sha") == sha:
+                return float(f["bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpus):
+        self.gpus = gpus
+        self.proc = None
+        self.out = os.path.join("/tmp", f"fa_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "50", "-i", ",".join(str(g) for g in self.gpus)],
+                                         stdout=open(self.out, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.out):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+                for n, v in zip(names, f[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+            os.remove(self.out)
+        except Exception:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+_CPU_WORKLOAD = []
+
+
+def cpu_oracle_sample(budget_s=12.0, max_heads=64, prefix=None):
+    """Time the fp64 oracle on whole (batch, head) problems of the workload until budget_s is spent."""
+    import oracle
+    from exact_tiled_attention_41_b200 import workloads as W
+
+    if not _CPU_WORKLOAD:
+        _CPU_WORKLOAD.append(W.dense_prefill(seed=0))
+    w = _CPU_WORKLOAD[0]
+    t = w.tensors
+    S = prefix or w.meta["Sq"]
+    q = t["q"][:, :S].double().numpy()
+    k = t["k"][:, :S].double().numpy()
+    v = t["v"][:, :S].double().numpy()
+    do = t["do"][:, :S].double().numpy()
+    mask = oracle.allowed_mask(S, S, True)
+    flops, heads = 0.0, 0
+    t0 = time.perf_counter()
+    for h in range(max_heads):
+        b, hh = divmod(h, w.meta["Hq"])
+        oracle.head_forward(q[b, :, hh], k[b, :, hh], v[b, :, hh], w.scale, mask)
+        oracle.head_backward(q[b, :, hh], k[b, :, hh], v[b, :, hh], do[b, :, hh], w.scale, mask)
+        flops += 3.5 * fwd_flops(1, 1, S, S, 128, True)
+        heads += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return flops, dt, heads, S
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        n = max((i.get("num_threads", 0) for i in info if i.get("user_api") == "blas"), default=0)
+        if n:
+            return n
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ---------------------------------------------------------------------------------------------- reference arm
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    # each step: fp64 oracle forward + backward of one (batch, head) problem on the first `prefix`
+    # tokens of the causal workload (rows there see exactly the same keys as in the full problem)
+    prefix = 512 if (args.steps + args.warmup) <= 400 else 256
+    for _ in range(args.warmup):
+        cpu_oracle_sample(budget_s=0.0, max_heads=1, prefix=prefix)
+    tot_flops, tot_dt = 0.0, 0.0
+    for _ in range(args.steps):
+        f, dt, _, _ = cpu_oracle_sample(budget_s=0.0, max_heads=1, prefix=prefix)
+        tot_flops += f
+        tot_dt += dt
+    value = tot_flops / tot_dt / 1e12
+    cores = cpu_threads()
+    sample = f"per step: fp64 oracle fwd+bwd of one (batch, head) causal problem on the first {prefix} tokens"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_dt / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": dict(WORKLOAD, parallelism="replicas"),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------------------------- our arm
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from exact_tiled_attention_41_b200 import abi, attention as A, workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    abi.load()
+    pk, pk_kind = peaks()
+
+    w = W.dense_prefill(seed=rank)
+    B, S, H, D = 4, 2048, 16, 128
+    t = {n: x.to(dev) for n, x in w.tensors.items()}
+    q, k, v, do = t["q"], t["k"], t["v"], t["do"]
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = abi.fa_bwd_workspace_size(B, H, H, S, S, D)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+    scale = w.scale
+    ff = fwd_flops(B, H, S, S, D, True)
+    step_flops = 3.5 * ff
+
+    def step():
+        st = abi.fa_fwd(q, k, v, out, lse, B, H, H, S, S, D, scale, 1, None, 0, stream)
+        st |= abi.fa_bwd(q, k, v, out, do, lse, dq, dk, dv, B, H, H, S, S, D, scale, 1, ws, ws_bytes, stream)
+        return st
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        if step() != 0:
+            raise RuntimeError("launch failed in warm-up")
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+
+    sampler = ClockSampler(list(range(world)) if world > 1 else [local_rank]) if local_rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    abi.fa_profile_begin(1)
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    abi.fa_profile_begin(0)
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    _, n_f, ms_f = abi.fa_profile_read(abi.FA_KERNEL_FWD)
+    _, n_b, ms_b = abi.fa_profile_read(abi.FA_KERNEL_BWD)
+    if world > 1:
+        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms = float(tt.item())
+    if abi.fa_get_device_status() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout during the timed region")
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+    # ----------------------------------------------------------------- end to end through the public API
+    e2e_steps = min(args.steps, 30)
+    pin = {n: x.cpu().pin_memory() for n, x in w.tensors.items()}
+    host_out = {n: torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
+                for n, x in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    h2d = sum(x.numel() * x.element_size() for x in pin.values())
+    d2h = sum(x.numel() * x.element_size() for x in host_out.values())
+
+    def e2e_step():
+        dq_ = {n: x.to(dev, non_blocking=True) for n, x in pin.items()}
+        o_, l_ = A.flash_attn_func(dq_["q"], dq_["k"], dq_["v"], scale, True)
+        g = A.flash_attn_backward(dq_["do"], dq_["q"], dq_["k"], dq_["v"], o_, l_, scale, True)
+        for n, x in zip(("out", "lse", "dq", "dk", "dv"), (o_, l_) + tuple(g)):
+            host_out[n].copy_(x, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+
+    extras = {}
+    if world == 1 and not args.no_extras:
+        extras = measure_extras(torch, abi, A, W, dev, pk)
+
+    if rank != 0:
+        return 0
+    peak_t = pk["bf16_tflops"]
+    bwd_ms = ms_b / max(n_b, 1)
+    fwd_ms = ms_f / max(n_f, 1)
+    bwd_tf = 2.5 * ff / (bwd_ms * 1e-3) / 1e12
+    fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
+    traffic = traffic_record("bwd_kernel", "exact_tiled_attention_41_b200/csrc/bwd.cu")
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(WORKLOAD, global_batch=4 * world, parallelism="replicas" if world > 1 else "single",
+                       l2="flushed before every step (256 MiB write, outside the per-step events)"),
+        "roofline": {"bound": "tensor", "kernel": "bwd_kernel (backward main)", "achieved": bwd_tf,
+                     "peak": peak_t, "unit": "TFLOP/s", "frac": bwd_tf / peak_t, "traffic": traffic,
+                     "peak_source": f"{pk_kind} bf16_tflops (burst)",
+                     "algorithmic_flops_per_launch": 2.5 * ff, "avg_launch_ms": bwd_ms, "launches": n_b},
+        "parts": {
+            "fwd_kernel": {"tflops": fwd_tf, "avg_launch_ms": fwd_ms, "launches": n_f,
+                           "frac_of_measured_peak": fwd_tf / peak_t, "frac_of_spec_2250": fwd_tf / 2250.0},
+            "bwd_kernel": {"tflops": bwd_tf, "avg_launch_ms": bwd_ms, "launches": n_b,
+                           "frac_of_measured_peak": bwd_tf / peak_t, "frac_of_spec_2250": bwd_tf / 2250.0},
+            "step_frac_of_measured_peak": value / world / peak_t,
+        },
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms, "api": "attention.flash_attn_func + flash_attn_backward, pinned host buffers"},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    if extras:
+        line["extras"] = extras
+    if world == 1 and not args.no_cpu_baseline:
+        f, dt, heads, Sx = cpu_oracle_sample(budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                                "sample": f"fp64 oracle fwd+bwd of {heads} whole (batch, head) problems of the "
+                                          f"workload (S={Sx}), {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def measure_extras(torch, abi, A, W, dev, pk):
+    """Other workloads, timed with CUDA events on the launching stream (not part of the step)."""
+    res = {}
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, iters):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    # long-context GQA: B=2, Hq=32, Hkv=8, S=8192, D=128, causal (inputs > L2)
+    w = W.gqa_long(seed=0)
+    t = {n: x.to(dev) for n, x in w.tensors.items()}
+    B, S, Hq, Hkv, D = 2, 8192, 32, 8, 128
+    out = torch.empty_like(t["q"])
+    lse = torch.empty((B, Hq, S), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+    nb = abi.fa_bwd_workspace_size(B, Hq, Hkv, S, S, D)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    ff = fwd_flops(B, Hq, S, S, D, True)
+    fms = timed(lambda: abi.fa_fwd(t["q"], t["k"], t["v"], out, lse, B, Hq, Hkv, S, S, D, w.scale, 1, None, 0,
+                                   stream), 5)
+    bms = timed(lambda: abi.fa_bwd(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, B, Hq, Hkv, S, S, D,
+                                   w.scale, 1, ws, nb, stream), 3)
+    res["gqa_long_B2_Hq32_Hkv8_S8192_D128_causal"] = {
+        "fwd_ms": fms, "fwd_tflops": ff / fms / 1e9, "bwd_ms": bms, "bwd_tflops": 2.5 * ff / bms / 1e9,
+        "fwd_frac_of_measured_peak": ff / fms / 1e9 / pk["bf16_tflops"],
+        "bwd_frac_of_measured_peak": 2.5 * ff / bms / 1e9 / pk["bf16_tflops"]}
+    del t, out, lse, dq, dk, dv, ws
+
+    # varlen packed batch, D = 64 and 256 (forward; backward for D = 64)
+    for D in (64, 256):
+        w = W.varlen_packed(D, seed=0)
+        t = {n: x.to(dev) for n, x in w.tensors.items()}
+        m = w.meta
+        lens = (w.tensors["cu_q"][1:] - w.tensors["cu_q"][:-1]).tolist()
+        ff = 4.0 * 0.5 * m["Hq"] * D * sum(L * L for L in lens)
+        out = torch.empty_like(t["q"])
+        lse = torch.empty((m["Hq"], m["total_q"]), dtype=torch.float32, device=dev)
+        fms = timed(lambda: abi.fa_varlen_fwd(t["q"], t["k"], t["v"], out, lse, t["cu_q"], t["cu_k"], 16, m["max_q"],
+                                              m["max_k"], m["total_q"], m["total_k"], 16, 16, D, w.scale, 1, None, 0,
+                                              stream), 5)
+        r = {"fwd_ms": fms, "fwd_tflops": ff / fms / 1e9, "total_tokens": m["total_q"]}
+        if D == 64:
+            dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+            nb = abi.fa_varlen_bwd_workspace_size(16, m["total_q"], m["total_k"], 16, 16, D)
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+            bms = timed(lambda: abi.fa_varlen_bwd(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, t["cu_q"],
+                                                  t["cu_k"], 16, m["max_q"], m["max_k"], m["total_q"], m["total_k"], 16,
+                                                  16, D, w.scale, 1, ws, nb, stream), 3)
+            r.update(bwd_ms=bms, bwd_tflops=2.5 * ff / bms / 1e9)
+        res[f"varlen_16seq_H16_D{D}_causal"] = r
+        del t
+
+    # KV-cache decode: B=64, Hq=32, Hkv=8, cache lengths U[1024, 16384], capacity 16384, D=128
+    w = W.decode(seed=0, nan_guard=False, device=str(dev))
+    t = w.tensors
+    lens = t["cache_seqlens"].to(dev)
+    B, Hq, Hkv, D, cap = 64, 32, 8, 128, 16384
+    out = torch.empty_like(t["q"])
+    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=dev)
+    nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, 1, cap, D, 0)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+    kv_bytes = float(w.tensors["cache_seqlens"].sum().item()) * Hkv * D * 2 * 2
+    alg_bytes = kv_bytes + 2 * t["q"].numel() * 2
+    abi.fa_profile_begin(1)
+    dms = timed(lambda: abi.fa_fwd_kvcache(t["q"], t["k_cache"], t["v_cache"], lens, out, lse, B, Hq, Hkv, 1, cap, D,
+                                           w.scale, 0, 0, ws, nb, stream), 10)
+    abi.fa_profile_begin(0)
+    _, n_s, ms_s = abi.fa_profile_read(abi.FA_KERNEL_DECODE)
+    split_ms = ms_s / max(n_s, 1)
+    res["decode_B64_Hq32_Hkv8_cap16384_D128"] = {
+        "ms": dms, "gbs": alg_bytes / dms / 1e6, "frac_of_measured_hbm": alg_bytes / dms / 1e6 / pk["hbm_gbs"],
+        "split_kernel_ms": split_ms, "split_kernel_gbs": kv_bytes / split_ms / 1e6,
+        "algorithmic_bytes": alg_bytes}
+    del t, w
+    torch.cuda.empty_cache()
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1 and dist.is_initialized():
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -66,12 +66,15 @@ int fa_profile_begin(int enable) {
             r.created = 0;
         }
     }
-    for (auto& r : g_rec) {
-        r.count = 0;
-        r.pending = false;
+    if (enable) {
+        // a new recording session starts empty; stopping keeps the records for fa_profile_read
+        for (auto& r : g_rec) {
+            r.count = 0;
+            r.pending = false;
+        }
+        g_device = dev;
     }
     g_enabled = enable != 0;
-    if (enable) g_device = dev;
     return FA_OK;
 }
 

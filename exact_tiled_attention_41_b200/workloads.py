@@ -33,7 +33,7 @@ class Workload:
 
 
 def _randn(g, shape):
-    return torch.randn(shape, generator=g, dtype=torch.float32).to(torch.bfloat16)
+    return torch.randn(shape, generator=g, dtype=torch.float32, device=g.device).to(torch.bfloat16)
 
 
 def dense(B, Sq, Sk, Hq, Hkv, D, causal, seed=0, with_grad=True, name=None) -> Workload:
@@ -78,21 +78,26 @@ def varlen_random(num_seqs, lo, hi, H, D, causal, seed=0, with_grad=True, name=N
     return varlen(lens, lens, H, H, D, causal, seed, with_grad, name, g=g)
 
 
-def kvcache(B, Hq, Hkv, D, capacity, lo, hi, seed=0, Sq=1, nan_guard=True, name=None, lengths=None) -> Workload:
+def kvcache(B, Hq, Hkv, D, capacity, lo, hi, seed=0, Sq=1, nan_guard=True, name=None, lengths=None,
+            device="cpu") -> Workload:
     """Contiguous cache (B, capacity, Hkv, D); rows >= cache_seqlens[b] hold NaN guards.
 
     Only the valid rows are drawn from the generator (K for every batch row,
     then V for every batch row), so the guard rows cost no random numbers.
+    Lengths always come from the CPU generator; ``device="cuda"`` draws the
+    tensors with a CUDA generator of the same seed (faster for multi-GB caches).
     """
     g = torch.Generator("cpu").manual_seed(seed)
     if lengths is None:
         lens = torch.randint(lo, hi + 1, (B,), generator=g, dtype=torch.int64)
     else:
         lens = torch.as_tensor(lengths, dtype=torch.int64)
+    if device != "cpu":
+        g = torch.Generator(device).manual_seed(seed)
     q = _randn(g, (B, Sq, Hq, D))
     fill = BF16_NAN if nan_guard else 0.0
-    kc = torch.full((B, capacity, Hkv, D), fill, dtype=torch.bfloat16)
-    vc = torch.full((B, capacity, Hkv, D), fill, dtype=torch.bfloat16)
+    kc = torch.full((B, capacity, Hkv, D), fill, dtype=torch.bfloat16, device=device)
+    vc = torch.full((B, capacity, Hkv, D), fill, dtype=torch.bfloat16, device=device)
     for b in range(B):
         L = int(lens[b])
         kc[b, :L] = _randn(g, (L, Hkv, D))
@@ -125,7 +130,7 @@ def varlen_packed(D: int, seed=0) -> Workload:
     return varlen_random(16, 128, 4096, 16, D, True, seed, name=f"varlen_16seq_L128-4096_H16_D{D}_causal")
 
 
-def decode(seed=0, nan_guard=True) -> Workload:
+def decode(seed=0, nan_guard=True, device="cpu") -> Workload:
     """B=64, Hq=32, Hkv=8, Sq=1, cache lengths uniform in [1024, 16384], capacity 16384, D=128."""
     return kvcache(64, 32, 8, 128, 16384, 1024, 16384, seed, 1, nan_guard,
-                   name="decode_B64_Hq32_Hkv8_cap16384_D128")
+                   name="decode_B64_Hq32_Hkv8_cap16384_D128", device=device)
