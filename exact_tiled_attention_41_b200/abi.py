@@ -30,6 +30,7 @@ EXPORTS = (
     "fa_fwd_kvcache", "fa_fwd_kvcache_workspace_size", "fa_status_string", "fa_get_device_status",
     "fa_set_wait_timeout_ns", "fa_debug_wait_timeout_selftest", "fa_debug_umma_selftest",
     "fa_profile_begin", "fa_profile_read",
+    "fa_fwd_kvcache_noalloc", "fa_fwd_kvcache_noalloc_scratch_bytes",
 )
 
 FA_KERNEL_FWD = 0
@@ -60,6 +61,8 @@ _SIGS = {
     "fa_debug_umma_selftest": (_I, [_P, _P, _P, _I, _P]),
     "fa_profile_begin": (_I, [_I]),
     "fa_profile_read": (_I, [_I, ctypes.POINTER(_I), ctypes.POINTER(_F)]),
+    "fa_fwd_kvcache_noalloc": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P]),
+    "fa_fwd_kvcache_noalloc_scratch_bytes": (_Z, []),
 }
 
 _lib = None
@@ -190,3 +193,15 @@ def fa_profile_read(kernel_id: int):
     ms = _F(0.0)
     st = load().fa_profile_read(int(kernel_id), ctypes.byref(n), ctypes.byref(ms))
     return st, n.value, ms.value
+
+
+def fa_fwd_kvcache_noalloc(q, k_cache, v_cache, cache_seqlens, out, lse, B, Hq, Hkv, Sq, cache_capacity, D,
+                           softmax_scale, causal, num_splits, stream=None) -> int:
+    """Decode for callers that cannot allocate: scratch lives in an array inside the library."""
+    return load().fa_fwd_kvcache_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens), _ptr(out),
+                                         _ptr(lse), B, Hq, Hkv, Sq, cache_capacity, D, float(softmax_scale),
+                                         int(bool(causal)), int(num_splits), _stream(stream))
+
+
+def fa_fwd_kvcache_noalloc_scratch_bytes() -> int:
+    return load().fa_fwd_kvcache_noalloc_scratch_bytes()

@@ -154,6 +154,34 @@ FA_API int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cach
                    float softmax_scale, int causal, int num_splits,
                    void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
+/* ------------------------------------------------------------------------- KV-cache decode without caller memory
+ * fa_fwd_kvcache_noalloc: the same computation as fa_fwd_kvcache, for callers
+ * that cannot allocate device memory when they decode -- for example code that
+ * runs while a CUDA graph is being captured and must not grow a memory pool,
+ * or a plugin / runtime that only receives the tensors it owns.  The source
+ * pages have no counterpart of this entry point; it is an interface addition.
+ *
+ * The per-split partial results live in one array compiled into the library
+ * (fa_fwd_kvcache_noalloc_scratch_bytes() bytes, 16 MiB).  Every GPU that loads
+ * the library holds that array until the process exits.  The caller still
+ * passes q, the caches, cache_seqlens, out and (optionally) lse exactly as for
+ * fa_fwd_kvcache; no workspace argument, and nothing is allocated or freed.
+ *   - The first call on a device looks up the array's device address there
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU (other streams,
+ *     other host threads) race on it and must be serialised by the caller.
+ *     Nothing in it needs to start at zero; each call writes what it reads.
+ *   - With num_splits = 0 the split is chosen as for fa_fwd_kvcache and made
+ *     coarser until the partials fit.  If they cannot fit (an explicit
+ *     num_splits too large, or B * Hq * (D + 1) * 4 bytes beyond the array),
+ *     the call returns FA_ERR_WORKSPACE and launches nothing.
+ */
+FA_API size_t fa_fwd_kvcache_noalloc_scratch_bytes(void);
+FA_API int fa_fwd_kvcache_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                  const int32_t* cache_seqlens, void* out, float* lse,
+                                  int B, int Hq, int Hkv, int Sq, int cache_capacity, int D,
+                                  float softmax_scale, int causal, int num_splits, fa_stream_t stream);
+
 /* ------------------------------------------------------------------------- helpers
  * fa_status_string: static English text for a status code (never NULL).
  */
