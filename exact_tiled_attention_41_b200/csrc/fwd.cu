@@ -101,7 +101,13 @@ struct FwdCfg {
     static constexpr uint32_t KV_BYTES = BK * D * 2;
     static constexpr int NUM_BARS = 5 * NQ + 4 * KST;
     static constexpr size_t SMEM = 1024 + NQ * Q_BYTES + 2 * KST * KV_BYTES + NUM_BARS * 8 + 16;
-    static constexpr int THREADS = (4 * NQ + 2) * 32;
+    // NQ softmax warpgroups + one warpgroup holding the producer warp, the MMA warp and two idle warps
+    static constexpr int THREADS = (4 * NQ + 4) * 32;
+    // register split with setmaxnreg (NQ = 2): launch at 168 per thread (384 x 168 = 64512),
+    // the producer/MMA warpgroup drops to 72 and the two softmax warpgroups rise to 216:
+    // 2 x 128 x 216 + 128 x 72 = 64512.  The host checks the launch count before the first launch.
+    static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, OTHER_REGS = 72;
+    static_assert(NQ != 2 || 2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
     static constexpr uint32_t S_COL(int i) { return i * BK; }
     static constexpr uint32_t O_COL(int i) { return NQ * BK + i * D; }
     static_assert(NQ * BK + NQ * D <= 512, "tensor memory budget");
@@ -170,7 +176,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const Watch w{abort_flag, p.status, p.timeout_ns};
-
+    // The last warpgroup (producer, MMA issuer, two idle warps) gives registers to the softmax warpgroups;
+    // each setmaxnreg is executed by all four warps of its warpgroup at the same instruction.
+    if (warp >= 4 * NQ) {
+    if constexpr (NQ == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
     if (warp == PRODUCER) {
         if (lane == 0) {
             uint32_t kv_it = 0, q_it = 0;
@@ -287,7 +296,9 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             }
         }
         __syncwarp();
+    }
     } else {
+        if constexpr (NQ == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::SOFTMAX_REGS));
         // ------------------------------------------------------------- softmax warpgroups
         const int i = warp >> 2;
         const int wq = warp & 3;
@@ -323,29 +334,24 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                 tc_fence_after();
                 float s[BK];
                 {
-                    uint32_t ra[32];
+                    // the whole row in one round trip: BK/32 loads, one wait
+                    uint32_t* sr = reinterpret_cast<uint32_t*>(s);
 #pragma unroll
-                    for (int cc = 0; cc < BK / 32; ++cc) {
-                        tmem_ld32(tS + cc * 32, ra);
-                        tmem_ld_wait_tie(ra);
+                    for (int cc = 0; cc < BK / 32; ++cc)
+                        tmem_ld32(tS + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(sr + cc * 32));
+                    tmem_ld_wait_tie(*reinterpret_cast<uint32_t(*)[32]>(sr));
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) s[cc * 32 + e] = __uint_as_float(ra[e]);
-                    }
+                    for (int cc = 1; cc < BK / 32; ++cc) reg_tie(*reinterpret_cast<uint32_t(*)[32]>(sr + cc * 32));
                 }
                 const int kbase = j * BK;
                 if (__any_sync(0xffffffffu, kbase + BK - 1 > key_lim)) {
 #pragma unroll
                     for (int c = 0; c < BK; ++c) s[c] = (kbase + c <= key_lim) ? s[c] : -INFINITY;
                 }
-                float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+                float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
-                for (int c = 4; c < BK; c += 4) {
-                    mx0 = fmaxf(mx0, s[c]);
-                    mx1 = fmaxf(mx1, s[c + 1]);
-                    mx2 = fmaxf(mx2, s[c + 2]);
-                    mx3 = fmaxf(mx3, s[c + 3]);
-                }
-                const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+                for (int c = 4; c < BK; c += 2) mx[(c >> 1) & 3] = max3f(mx[(c >> 1) & 3], s[c], s[c + 1]);
+                const float mt = max3f(mx[0], mx[1], fmaxf(mx[2], mx[3]));
                 const bool need = (mt - m_ref) * c2 > kDeferLog2;   // NaN (both -inf) -> false
                 if (__any_sync(0xffffffffu, need)) {
                     const float m_new = fmaxf(m_ref, mt);
@@ -357,12 +363,17 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                         if (__all_sync(0xffffffffu, ok)) {
                             tc_fence_after();
                             uint32_t ro[32];
+                            const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll 1
                             for (int cc = 0; cc < D / 32; ++cc) {
                                 tmem_ld32(tO + cc * 32, ro);
                                 tmem_ld_wait_tie(ro);
 #pragma unroll
-                                for (int e = 0; e < 32; ++e) ro[e] = __float_as_uint(__uint_as_float(ro[e]) * alpha);
+                                for (int e = 0; e < 32; e += 2) {
+                                    const float2 v = fmul2(make_float2(__uint_as_float(ro[e]), __uint_as_float(ro[e + 1])), a2);
+                                    ro[e] = __float_as_uint(v.x);
+                                    ro[e + 1] = __float_as_uint(v.y);
+                                }
                                 tmem_st32(tO + cc * 32, ro);
                             }
                             tmem_st_wait();
@@ -375,21 +386,25 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     m_ref = m_new;
                 }
                 const float ms = (m_ref == -INFINITY) ? 0.f : m_ref * c2;
-                float sum0 = 0.f, sum1 = 0.f;
+                const float2 c2v = make_float2(c2, c2), nms = make_float2(-ms, -ms);
+                float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int half = 0; half < BK / 64; ++half) {
                     uint32_t pk[32];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
-                        const float a = ex2_approx(fmaf(s[half * 64 + 2 * e], c2, -ms));
-                        const float b = ex2_approx(fmaf(s[half * 64 + 2 * e + 1], c2, -ms));
-                        sum0 += a;
-                        sum1 += b;
-                        pk[e] = pack_bf16x2(a, b);
+                        // exp(scale * s - scale * m) as exp2 of one fused multiply-add per pair
+                        const float2 x = ffma2(make_float2(s[half * 64 + 2 * e], s[half * 64 + 2 * e + 1]), c2v, nms);
+                        const float2 p2 = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        if (e & 1) sum1 = fadd2(sum1, p2); else sum0 = fadd2(sum0, p2);
+                        pk[e] = pack_bf16x2(p2.x, p2.y);
                     }
                     tmem_st32(tS + half * 32, pk);
                 }
-                l += sum0 + sum1;
+                {
+                    const float2 sm = fadd2(sum0, sum1);
+                    l += sm.x + sm.y;
+                }
                 tmem_st_wait();
                 tc_fence_before();
                 mbar_arrive(p_full(i));
@@ -406,9 +421,12 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                 tmem_ld32(tO + cc * 32, ro);
                 tmem_ld_wait_tie(ro);
                 uint32_t pk[16];
+                const float2 il = make_float2(inv_l, inv_l);
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    pk[e] = pack_bf16x2(__uint_as_float(ro[2 * e]) * inv_l, __uint_as_float(ro[2 * e + 1]) * inv_l);
+                for (int e = 0; e < 16; ++e) {
+                    const float2 v = fmul2(make_float2(__uint_as_float(ro[2 * e]), __uint_as_float(ro[2 * e + 1])), il);
+                    pk[e] = pack_bf16x2(v.x, v.y);
+                }
                 if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
@@ -474,6 +492,12 @@ static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, 
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
             cudaSuccess)
             return 5;
+        if (NQ == 2) {
+            // the setmaxnreg split assumes exactly LAUNCH_REGS per thread at launch; with fewer the
+            // increase could never be granted, so refuse to launch instead
+            cudaFuncAttributes fa_attr;
+            if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess || fa_attr.numRegs != C::LAUNCH_REGS) return 2;
+        }
         attr_set[dev.id & 63] = true;
     }
     const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
