@@ -15,17 +15,20 @@
 //      is (sequence, KV head, 128-key tile); it loops over the 128-row query
 //      tiles of every query head that reads the KV head (so dK and dV of GQA
 //      need no atomics) and, for causal masks, only over query tiles that can
-//      see the key tile.  Roles:
-//        warps 0-3  compute: thread = key row; P^T, dS^T from S^T and dP^T in
-//                   tensor memory; dK / dV epilogue
-//        warps 4-7  dQ: thread = query row; reads the dQ tile from tensor memory
-//                   and adds it to the fp32 accumulator (vector atomics)
-//        warp 8     producer: K, V once per unit; Q, dO tiles (TMA) and the
-//                   tile's LSE2 / Delta (plain loads) through a 2-stage ring
-//        warp 9     tensor memory and every tcgen05 MMA:
-//                   S^T = K Q^T, dP^T = V dO^T              (K-major x K-major)
-//                   dV += P^T dO, dK += dS^T Q               (tensor-memory A)
-//                   dQ = dS K                                (N-major x N-major)
+//      see the key tile.  Roles (16 warps, registers redistributed with setmaxnreg):
+//        warps 0-7   two compute warpgroups, thread = key row, each owning 64 of
+//                    the 128 query columns: P^T, dS^T from S^T and dP^T in tensor
+//                    memory (written back as bf16, dS^T also to shared memory);
+//                    dV (warpgroup 0) / dK (warpgroup 1) epilogue
+//        warps 8-11  dQ: thread = query row; reads the dQ tile from tensor memory
+//                    and adds it to the fp32 accumulator (vector atomics)
+//        warp 12     producer: K, V once per unit; Q, dO tiles (TMA) and the
+//                    tile's LSE2 / Delta (plain loads) through a 2-stage ring
+//        warp 13     tensor memory and every tcgen05 MMA, in this order per tile:
+//                    S^T = K Q^T, dP^T = V dO^T              (K-major x K-major)
+//                    dQ = dS K into the columns of S^T / dP^T left free by the
+//                    bf16 P^T / dS^T, so the dQ read-out overlaps   (N-major x N-major)
+//                    dV += P^T dO, dK += dS^T Q               (tensor-memory A)
 //   3. convert: dQ = bf16(scale * dQacc).
 #include "internal.h"
 #include "sm100.cuh"
@@ -93,22 +96,31 @@ __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
 
 template <int D>
 struct BwdCfg {
-    static constexpr int BM = 128, BN = 128, ST = 2;
+    static constexpr int ST = 2;
     static constexpr int NCHUNK = D / 64;
     static constexpr uint32_t T_BYTES = 128 * D * 2;      // one 128-row tile of K, V, Q or dO
-    static constexpr uint32_t DS_BYTES = 128 * 128 * 2;   // dS^T [key][query]
+    static constexpr uint32_t DS_BYTES = 128 * 128 * 2;   // dS^T [key][query], two 64-query boxes
     // layout: K | V | Q[ST] | dO[ST] | dS | LSE2[ST][128] | Delta[ST][128] | barriers
     static constexpr uint32_t OFF_K = 0, OFF_V = T_BYTES, OFF_Q = 2 * T_BYTES, OFF_DO = (2 + ST) * T_BYTES,
                               OFF_DS = (2 + 2 * ST) * T_BYTES, OFF_STAT = OFF_DS + DS_BYTES,
                               OFF_BAR = OFF_STAT + 2 * ST * 128 * 4;
     static constexpr int NUM_BARS = 2 + 2 * ST + 5;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
+    // tensor memory: dV | dK | S^T | dP^T.  After the gradient step P^T and dS^T (bf16) occupy the
+    // low 64 columns of S^T and dP^T; dQ (fp32) is accumulated into their free high 64 columns.
     static constexpr uint32_t COL_DV = 0, COL_DK = D, COL_S = 2 * D, COL_DP = 2 * D + 128;
+    static constexpr uint32_t COL_DQ(int h) { return h == 0 ? COL_S + 64 : COL_DP + 64; }
     static_assert(2 * D + 256 <= 512, "tensor memory budget");
+    static_assert(D == 64 || D == 128, "dQ halves map onto the free columns for D <= 128");
+    // 16 warps: 0-7 two compute warpgroups (query columns 0-63 / 64-127), 8-11 dQ warpgroup,
+    // 12 producer, 13 MMA issuer, 14-15 idle.  Registers: launch at 128 per thread (512 x 128 = 65536);
+    // 2 x 128 x 184 + 128 x 64 + 128 x 72 = 64512.  The host checks the launch count.
+    static constexpr int THREADS = 512, LAUNCH_REGS = 128, COMPUTE_REGS = 184, DQ_REGS = 64, OTHER_REGS = 72;
+    static_assert(2 * 128 * COMPUTE_REGS + 128 * DQ_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                const __grid_constant__ BwdParams p) {
@@ -128,7 +140,7 @@ __global__ void __launch_bounds__(320, 1)
                    dq_empty = s_full + 24, dkv_full = s_full + 32;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int PRODUCER = 8, MMA = 9;
+    constexpr int PRODUCER = 12, MMA = 13;
 
     if ((smem_u32(smem) & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
         if (threadIdx.x == 0) atomicCAS(p.status, 0, 2);
@@ -138,11 +150,11 @@ __global__ void __launch_bounds__(320, 1)
         mbar_init(bars + 0, 1);
         mbar_init(bars + 1, 1);
         for (int s = 0; s < ST; ++s) {
-            mbar_init(bars + 2 + s, 33);
+            mbar_init(bars + 2 + s, 33);        // 32 producer lanes (statistics) + the TMA expect-tx arrival
             mbar_init(bars + 2 + ST + s, 1);
         }
         mbar_init(bars + 2 + 2 * ST + 0, 1);    // s_full
-        mbar_init(bars + 2 + 2 * ST + 1, 128);  // p_full
+        mbar_init(bars + 2 + 2 * ST + 1, 256);  // p_full: both compute warpgroups
         mbar_init(bars + 2 + 2 * ST + 2, 1);    // dq_full
         mbar_init(bars + 2 + 2 * ST + 3, 128);  // dq_empty
         mbar_init(bars + 2 + 2 * ST + 4, 1);    // dkv_full
@@ -166,228 +178,126 @@ __global__ void __launch_bounds__(320, 1)
     const Watch w{abort_flag, p.status, p.timeout_ns};
     const int G = p.group;
 
-    if (warp == PRODUCER) {
-        // ------------------------------------------------------------ producer (whole warp)
-        uint32_t unit_it = 0, q_it = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-            const BUnit t = decode_bunit(p, u);
-            if (t.skip || t.n_it == 0) continue;
-            if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
-            if (lane == 0) {
-                mbar_arrive_expect_tx(kv_full, 2 * C::T_BYTES);
-#pragma unroll
-                for (int c = 0; c < C::NCHUNK; ++c) {
-                    tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
-                                t.k_start + t.n0);
-                    tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
-                                t.k_start + t.n0);
-                }
-            }
-            ++unit_it;
-            for (int it = 0; it < t.n_it; ++it, ++q_it) {
-                const int g = it / t.n_m;
-                const int m0 = (t.m_start + it % t.n_m) * 128;
-                const int h = t.hk * G + g;
-                const int st = q_it % ST;
-                if (q_it >= ST && !mbar_wait(q_empty(st), ((q_it / ST) - 1) & 1, w)) { ok = false; break; }
-                // tile statistics; rows past the sequence get LSE2 = +inf (P = 0) and Delta = 0
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int qi = lane * 4 + e;
-                    const int row = m0 + qi;
-                    const bool in = row < t.Lq;
-                    const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
-                    sLSE[st * 128 + qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
-                    sDel[st * 128 + qi] = in ? __ldg(p.delta + idx) : 0.f;
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(q_full(st), 2 * C::T_BYTES);
-#pragma unroll
-                    for (int c = 0; c < C::NCHUNK; ++c) {
-                        tma_load_3d(smem_u32(smem + C::OFF_Q + st * C::T_BYTES + c * 128 * 128), &tmQ, q_full(st),
-                                    c * 64, h, t.q_start + m0);
-                        tma_load_3d(smem_u32(smem + C::OFF_DO + st * C::T_BYTES + c * 128 * 128), &tmDO, q_full(st),
-                                    c * 64, h, t.q_start + m0);
-                    }
-                }
-                mbar_arrive(q_full(st));
-            }
-        }
-        __syncwarp();
-    } else if (warp == MMA) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
-            constexpr uint32_t id_tn = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
-            constexpr uint32_t id_mm = idesc_bf16_f32(128, D, true, true);       // dQ
-            uint32_t unit_it = 0, q_it = 0, g_it = 0;
+    if (warp >= 12) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
+        if (warp == PRODUCER) {
+            // -------------------------------------------------------- producer (whole warp)
+            uint32_t unit_it = 0, q_it = 0;
             bool ok = true;
             for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
                 const BUnit t = decode_bunit(p, u);
                 if (t.skip || t.n_it == 0) continue;
-                if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
-                for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
-                    const int st = q_it % ST;
-                    if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
-                    if (g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
-                    tc_fence_after();
-                    const uint8_t* sq = smem + C::OFF_Q + st * C::T_BYTES;
-                    const uint8_t* sdo = smem + C::OFF_DO + st * C::T_BYTES;
+                if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(kv_full, 2 * C::T_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                        umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + o), 16, 1024),
-                                sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
+                    for (int c = 0; c < C::NCHUNK; ++c) {
+                        tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
+                        tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
                     }
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                        umma_ss(tmem + C::COL_DP, sdesc_sw128(smem_u32(smem + C::OFF_V + o), 16, 1024),
-                                sdesc_sw128(smem_u32(sdo + o), 16, 1024), id_kk, kk > 0);
-                    }
-                    umma_commit(s_full);
-                    if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
-                    tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 query rows
-                        const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                        umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8,
-                                sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
-                        umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8,
-                                sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
-                    }
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
-                        umma_ss(tmem + C::COL_S,
-                                sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
-                                sdesc_sw128(smem_u32(smem + C::OFF_K + kk * 16 * 128), 128 * 128, 1024), id_mm,
-                                kk > 0);
-                    }
-                    umma_commit(dq_full);
-                    umma_commit(q_empty(st));
                 }
-                if (!ok) break;
-                umma_commit(dkv_full);
-                umma_commit(kv_empty);
                 ++unit_it;
-            }
-        }
-        __syncwarp();
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ compute warpgroup (thread = key row)
-        const int r = warp * 32 + lane;
-        const uint32_t lb = tmem_lane_base(warp);
-        const float c2 = p.scale_log2;
-        uint32_t unit_it = 0, q_it = 0, g_it = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
-            const BUnit t = decode_bunit(p, u);
-            if (t.skip) continue;
-            const int kj = t.n0 + r;                 // key index inside the sequence
-            const bool kvalid = kj < t.Lk;
-            const size_t krow = (static_cast<size_t>(t.k_start) + kj) * p.Hkv + t.hk;
-            if (t.n_it == 0) {
-                if (kvalid) {
-                    const uint4 z = make_uint4(0, 0, 0, 0);
-                    for (int c = 0; c < D / 8; ++c) {
-                        reinterpret_cast<uint4*>(p.dk + krow * D)[c] = z;
-                        reinterpret_cast<uint4*>(p.dv + krow * D)[c] = z;
+                for (int it = 0; it < t.n_it; ++it, ++q_it) {
+                    const int g = it / t.n_m;
+                    const int m0 = (t.m_start + it % t.n_m) * 128;
+                    const int h = t.hk * G + g;
+                    const int st = q_it % ST;
+                    if (q_it >= ST && !mbar_wait(q_empty(st), ((q_it / ST) - 1) & 1, w)) { ok = false; break; }
+                    // tile statistics; rows past the sequence get LSE2 = +inf (P = 0) and Delta = 0
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int qi = lane * 4 + e;
+                        const int row = m0 + qi;
+                        const bool in = row < t.Lq;
+                        const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
+                        sLSE[st * 128 + qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
+                        sDel[st * 128 + qi] = in ? __ldg(p.delta + idx) : 0.f;
                     }
-                }
-                continue;
-            }
-            const int off = t.Lk - t.Lq;
-            for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
-                const int m0 = (t.m_start + it % t.n_m) * 128;
-                const int st = q_it % ST;
-                if (!mbar_wait(s_full, g_it & 1, w)) { ok = false; break; }
-                if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
-                tc_fence_after();
-                // key kj may be seen by query row qi iff kj <= qi + off  <=>  qi >= kj - off
-                const int qmin = p.causal ? kj - off - m0 : -0x40000000;   // first allowed local query column
-                const bool full_row = kvalid && qmin <= 0;
-                const bool any_mask = __any_sync(0xffffffffu, !full_row);
-                const float* lse_t = sLSE + st * 128;
-                const float* del_t = sDel + st * 128;
-                uint8_t* ds_row = smem + C::OFF_DS + r * 128;
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t sa[32], da[32];
-                    tmem_ld32(tmem + lb + C::COL_S + cc * 32, sa);
-                    tmem_ld32(tmem + lb + C::COL_DP + cc * 32, da);
-                    tmem_ld_wait_tie(sa);
-                    reg_tie(da);
-                    uint32_t pp[16], dd[16];
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(q_full(st), 2 * C::T_BYTES);
 #pragma unroll
-                    for (int e = 0; e < 32; e += 4) {
-                        const float4 l4 = *reinterpret_cast<const float4*>(lse_t + cc * 32 + e);
-                        const float4 d4 = *reinterpret_cast<const float4*>(del_t + cc * 32 + e);
-                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                        const float dv[4] = {d4.x, d4.y, d4.z, d4.w};
-                        float pv[4], sv[4];
-#pragma unroll
-                        for (int x = 0; x < 4; ++x) {
-                            float pr = ex2_approx(fmaf(__uint_as_float(sa[e + x]), c2, -lv[x]));
-                            if (any_mask) {
-                                const int qc = cc * 32 + e + x;
-                                pr = (kvalid && qc >= qmin) ? pr : 0.f;
-                            }
-                            pv[x] = pr;
-                            sv[x] = pr * (__uint_as_float(da[e + x]) - dv[x]);
+                        for (int c = 0; c < C::NCHUNK; ++c) {
+                            tma_load_3d(smem_u32(smem + C::OFF_Q + st * C::T_BYTES + c * 128 * 128), &tmQ, q_full(st),
+                                        c * 64, h, t.q_start + m0);
+                            tma_load_3d(smem_u32(smem + C::OFF_DO + st * C::T_BYTES + c * 128 * 128), &tmDO,
+                                        q_full(st), c * 64, h, t.q_start + m0);
                         }
-                        pp[e / 2] = pack_bf16x2(pv[0], pv[1]);
-                        pp[e / 2 + 1] = pack_bf16x2(pv[2], pv[3]);
-                        dd[e / 2] = pack_bf16x2(sv[0], sv[1]);
-                        dd[e / 2 + 1] = pack_bf16x2(sv[2], sv[3]);
                     }
-                    tmem_st16(tmem + lb + C::COL_S + cc * 16, pp);
-                    tmem_st16(tmem + lb + C::COL_DP + cc * 16, dd);
-                    // dS^T row r, query columns 32cc .. 32cc+31: 4 chunks of 16 bytes (128-byte swizzle)
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int chunk = cc * 4 + q4;               // 8 query columns per chunk
-                        const int box = chunk >> 3, cin = chunk & 7;
-                        *reinterpret_cast<uint4*>(ds_row + box * 128 * 128 + ((cin ^ (r & 7)) << 4)) =
-                            make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
-                    }
-                }
-                tmem_st_wait();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(p_full);
-            }
-            if (!ok) break;
-            // -------------------------------------------------- dK, dV epilogue
-            if (!mbar_wait(dkv_full, unit_it & 1, w)) { ok = false; break; }
-            ++unit_it;
-            tc_fence_after();
-#pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col = which == 0 ? C::COL_DV : C::COL_DK;
-                const float mul = which == 0 ? 1.f : p.scale;
-                __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + krow * D;
-#pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t ra[32];
-                    tmem_ld32(tmem + lb + col + cc * 32, ra);
-                    tmem_ld_wait_tie(ra);
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        pk[e] = pack_bf16x2(__uint_as_float(ra[2 * e]) * mul, __uint_as_float(ra[2 * e + 1]) * mul);
-                    if (kvalid) {
-                        uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                    }
+                    mbar_arrive(q_full(st));
                 }
             }
-            tc_fence_before();
+            __syncwarp();
+        } else if (warp == MMA) {
+            // -------------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
+                constexpr uint32_t id_tn = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
+                constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);      // dQ, 64 columns at a time
+                uint32_t unit_it = 0, q_it = 0, g_it = 0;
+                bool ok = true;
+                for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                    const BUnit t = decode_bunit(p, u);
+                    if (t.skip || t.n_it == 0) continue;
+                    if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
+                    for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
+                        const int st = q_it % ST;
+                        if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
+                        if (g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint8_t* sq = smem + C::OFF_Q + st * C::T_BYTES;
+                        const uint8_t* sdo = smem + C::OFF_DO + st * C::T_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+                            umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + o), 16, 1024),
+                                    sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+                            umma_ss(tmem + C::COL_DP, sdesc_sw128(smem_u32(smem + C::OFF_V + o), 16, 1024),
+                                    sdesc_sw128(smem_u32(sdo + o), 16, 1024), id_kk, kk > 0);
+                        }
+                        umma_commit(s_full);
+                        if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
+                        tc_fence_after();
+                        // dQ = dS K first, into the free high columns, so its read-out overlaps dV / dK
+#pragma unroll
+                        for (int hh = 0; hh < D / 64; ++hh) {
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
+                                umma_ss(tmem + C::COL_DQ(hh),
+                                        sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
+                                        sdesc_sw128(smem_u32(smem + C::OFF_K + hh * 128 * 128 + kk * 16 * 128),
+                                                    128 * 128, 1024),
+                                        id_dq, kk > 0);
+                            }
+                        }
+                        umma_commit(dq_full);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 query rows
+                            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                            umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8,
+                                    sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8,
+                                    sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                        }
+                        umma_commit(q_empty(st));
+                    }
+                    if (!ok) break;
+                    umma_commit(dkv_full);
+                    umma_commit(kv_empty);
+                    ++unit_it;
+                }
+            }
+            __syncwarp();
         }
-    } else {
+    } else if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::DQ_REGS));
         // ------------------------------------------------------------ dQ warpgroup (thread = query row)
-        const int wq = warp - 4;
+        const int wq = warp - 8;
         const int r = wq * 32 + lane;
         const uint32_t lb = tmem_lane_base(wq);
         uint32_t g_it = 0;
@@ -407,20 +317,148 @@ __global__ void __launch_bounds__(320, 1)
 #pragma unroll 1
                 for (int cc = 0; cc < D / 32; ++cc) {
                     uint32_t ra[32];
-                    tmem_ld32(tmem + lb + C::COL_S + cc * 32, ra);
+                    tmem_ld32(tmem + lb + C::COL_DQ(cc >> 1) + (cc & 1) * 32, ra);
                     tmem_ld_wait_tie(ra);
                     if (valid) {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const float4 v = make_float4(__uint_as_float(ra[4 * e]), __uint_as_float(ra[4 * e + 1]),
-                                                         __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3]));
-                            atomicAdd(acc + static_cast<size_t>(cc * 8 + e) * p.Tq, v);
-                        }
+                        for (int e = 0; e < 8; ++e)
+                            atomicAdd(acc + static_cast<size_t>(cc * 8 + e) * p.Tq,
+                                      make_float4(__uint_as_float(ra[4 * e]), __uint_as_float(ra[4 * e + 1]),
+                                                  __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3])));
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(dq_empty);
             }
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
+        // ------------------------------------------------------------ compute warpgroups (thread = key row)
+        const int gq = warp >> 2;                  // query columns [64 gq, 64 gq + 64)
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lb = tmem_lane_base(warp & 3);
+        const float c2 = p.scale_log2;
+        uint32_t unit_it = 0, q_it = 0, g_it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const BUnit t = decode_bunit(p, u);
+            if (t.skip) continue;
+            const int kj = t.n0 + r;                 // key index inside the sequence
+            const bool kvalid = kj < t.Lk;
+            const size_t krow = (static_cast<size_t>(t.k_start) + kj) * p.Hkv + t.hk;
+            __nv_bfloat16* gdst = (gq == 0 ? p.dv : p.dk) + krow * D;
+            if (t.n_it == 0) {
+                if (kvalid) {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(gdst)[c] = z;
+                }
+                continue;
+            }
+            const int off = t.Lk - t.Lq;
+            for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
+                const int m0 = (t.m_start + it % t.n_m) * 128;
+                const int st = q_it % ST;
+                bool got = mbar_wait(s_full, g_it & 1, w);
+                got = got && mbar_wait(q_full(st), (q_it / ST) & 1, w);
+                uint32_t sa[2][32], da[2][32];
+                if (__all_sync(0xffffffffu, got)) {
+                    tc_fence_after();
+                    tmem_ld32(tmem + lb + C::COL_S + 64 * gq, sa[0]);
+                    tmem_ld32(tmem + lb + C::COL_S + 64 * gq + 32, sa[1]);
+                    tmem_ld32(tmem + lb + C::COL_DP + 64 * gq, da[0]);
+                    tmem_ld32(tmem + lb + C::COL_DP + 64 * gq + 32, da[1]);
+                    tmem_ld_wait_tie(sa[0]);
+                    reg_tie(sa[1]);
+                    reg_tie(da[0]);
+                    reg_tie(da[1]);
+                } else {
+                    got = false;
+                }
+                // Both warpgroups hold their columns before either overwrites the low columns with
+                // P^T / dS^T.  Every compute thread passes this barrier once per iteration, also on abort,
+                // and all of them leave together if any wait gave up.
+                uint32_t all_got;
+                asm volatile(
+                    "{\n\t.reg .pred pa, pb;\n\tsetp.ne.u32 pa, %1, 0;\n\t"
+                    "bar.red.and.pred pb, 1, 256, pa;\n\tselp.u32 %0, 1, 0, pb;\n\t}\n"
+                    : "=r"(all_got)
+                    : "r"(static_cast<uint32_t>(got))
+                    : "memory");
+                if (!all_got) { ok = false; break; }
+                // key kj may be seen by query row qi iff kj <= qi + off  <=>  qi >= kj - off
+                const int qmin = p.causal ? kj - off - m0 : -0x40000000;   // first allowed local query column
+                const bool full_row = kvalid && qmin <= 64 * gq;
+                const bool any_mask = __any_sync(0xffffffffu, !full_row);
+                const float* lse_t = sLSE + st * 128 + 64 * gq;
+                const float* del_t = sDel + st * 128 + 64 * gq;
+                const float2 c2v = make_float2(c2, c2);
+                uint8_t* ds_row = smem + C::OFF_DS + gq * 128 * 128 + r * 128;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pp[16], dd[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 l4 = *reinterpret_cast<const float4*>(lse_t + half * 32 + e);
+                        const float4 d4 = *reinterpret_cast<const float4*>(del_t + half * 32 + e);
+#pragma unroll
+                        for (int x = 0; x < 4; x += 2) {
+                            const float la = x == 0 ? l4.x : l4.z, lbv = x == 0 ? l4.y : l4.w;
+                            const float dla = x == 0 ? d4.x : d4.z, dlb = x == 0 ? d4.y : d4.w;
+                            const float2 sv = make_float2(__uint_as_float(sa[half][e + x]), __uint_as_float(sa[half][e + x + 1]));
+                            const float2 dv = make_float2(__uint_as_float(da[half][e + x]), __uint_as_float(da[half][e + x + 1]));
+                            const float2 a = ffma2(sv, c2v, make_float2(-la, -lbv));
+                            float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                            if (any_mask) {
+                                const int qc = 64 * gq + half * 32 + e + x;
+                                pr.x = (kvalid && qc >= qmin) ? pr.x : 0.f;
+                                pr.y = (kvalid && qc + 1 >= qmin) ? pr.y : 0.f;
+                            }
+                            const float2 ds = fmul2(pr, fadd2(dv, make_float2(-dla, -dlb)));
+                            pp[(e + x) / 2] = pack_bf16x2(pr.x, pr.y);
+                            dd[(e + x) / 2] = pack_bf16x2(ds.x, ds.y);
+                        }
+                    }
+                    // P^T and dS^T of query columns [64 gq + 32 half, +32) -> packed columns [32 gq + 16 half, +16)
+                    tmem_st16(tmem + lb + C::COL_S + 32 * gq + 16 * half, pp);
+                    tmem_st16(tmem + lb + C::COL_DP + 32 * gq + 16 * half, dd);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int cin = half * 4 + q4;            // 16-byte chunk of the 64-query box row
+                        *reinterpret_cast<uint4*>(ds_row + ((cin ^ (r & 7)) << 4)) =
+                            make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
+                    }
+                }
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (!ok) break;
+            // -------------------------------------------------- epilogue: warpgroup 0 writes dV, 1 writes dK
+            if (!mbar_wait(dkv_full, unit_it & 1, w)) { ok = false; break; }
+            ++unit_it;
+            tc_fence_after();
+            const uint32_t col = gq == 0 ? C::COL_DV : C::COL_DK;
+            const float mul = gq == 0 ? 1.f : p.scale;
+            const float2 mul2 = make_float2(mul, mul);
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t ra[32];
+                tmem_ld32(tmem + lb + col + cc * 32, ra);
+                tmem_ld_wait_tie(ra);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float2 v = fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), mul2);
+                    pk[e] = pack_bf16x2(v.x, v.y);
+                }
+                if (kvalid) {
+                    uint4* o4 = reinterpret_cast<uint4*>(gdst + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+            tc_fence_before();
         }
     }
 
@@ -580,12 +618,15 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
             cudaSuccess)
             return 5;
+        // the setmaxnreg split assumes exactly LAUNCH_REGS per thread at launch
+        cudaFuncAttributes fa_attr;
+        if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess || fa_attr.numRegs != C::LAUNCH_REGS) return 2;
         set[dev.id & 63] = true;
     }
     const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
     if (grid > 0) {
         prof_before(1, stream);
-        kern<<<grid, 320, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
         prof_after(1, stream);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
