@@ -635,11 +635,31 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
 }
 
+// Head dim 256: same preprocess, then the half-head-dim kernel of bwd256.cu (which also converts dQ).
+static int run_bwd256(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
+                      void* dv, void* workspace, const Device& dev, cudaStream_t stream) {
+    constexpr int D = 256;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    float* dq_acc = static_cast<float*>(workspace);
+    float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + up(static_cast<size_t>(pr.Tq) * pr.Hq * D * 4));
+    float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + up(static_cast<size_t>(pr.Tq) * pr.Hq * 4));
+    const long long rows = static_cast<long long>(pr.Tq) * pr.Hq;
+    long long blocks = (rows + 7) / 8;
+    const long long cap = static_cast<long long>(dev.num_sms) * 16;
+    if (blocks > cap) blocks = cap;
+    bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta, dq_acc,
+        pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+    if (cudaPeekAtLastError() != cudaSuccess) return 5;
+    return launch_bwd256_main(pr, dout, lse2, delta, dq_acc, dq, dk, dv, dev, stream);
+}
+
 int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk, void* dv,
                void* workspace, const Device& dev, cudaStream_t stream) {
     switch (pr.D) {
         case 64: return run_bwd<64>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
         case 128: return run_bwd<128>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
+        case 256: return run_bwd256(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
         default: return 2;
     }
 }

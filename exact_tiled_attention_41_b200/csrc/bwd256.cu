@@ -1,0 +1,489 @@
+// bwd256.cu -- backward main kernel and dQ convert for head dim 256.
+//
+// Same mathematics as bwd.cu (recompute P from the stored LSE; dV = P^T dO,
+// dP = dO V^T, dS = P (dP - Delta), dQ = scale dS K, dK = scale dS^T Q), with a
+// tiling that fits tensor memory at D = 256: dV and dK of a 128-key tile would
+// take all 512 columns, so each work unit owns one half (128 columns) of the
+// head dimension of dV and dK.  The unit still contracts S^T = K Q^T and
+// dP^T = V dO^T over the full head dimension (the two halves recompute them),
+// and emits the matching half of dQ.  Query tiles are 64 rows so that K, V
+// (128 x 256 each), Q, dO (64 x 256) and dS^T fit shared memory.
+//   tensor memory: dV half [0,128) | dK half [128,256) | S^T [256,320) |
+//                  dP^T [320,384) | dQ^T half [384,448)
+//   dQ^T = K_half^T dS^T has the head dimension on the 128 lanes, so the dQ
+//   warpgroup's atomics cover 32 consecutive head-dim floats per warp and the
+//   accumulator is laid out [Hq][Tq][256].
+// Roles: warps 0-3 compute (thread = key row), 4-7 dQ (thread = head-dim row),
+// 8 producer, 9 MMA issuer, 10-11 idle; registers redistributed with setmaxnreg.
+#include "internal.h"
+#include "sm100.cuh"
+
+#include <math.h>
+
+namespace fa {
+
+namespace {
+
+constexpr int D = 256;
+
+struct B256Params {
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* dq_acc;          // [Hq][Tq][256]
+    const float* lse2;      // [Hq][Tq]
+    const float* delta;     // [Hq][Tq]
+    const int32_t* cu_q;
+    const int32_t* cu_k;
+    int num_seqs, Sq, Sk, Tq, Tk, Hq, Hkv, group;
+    int num_units;
+    float scale, scale_log2;
+    int causal;
+    unsigned long long timeout_ns;
+    int* status;
+};
+
+struct U256 {
+    int b, hk, hh, q_start, k_start, Lq, Lk, n0, m_start, n_m, n_it;
+    bool skip;
+};
+
+__device__ __forceinline__ U256 decode_u256(const B256Params& p, int u) {
+    U256 t;
+    const int per_n = p.num_seqs * p.Hkv * 2;
+    const int n = u / per_n;            // key tile; the first tiles have the most work under a causal mask
+    int r = u % per_n;
+    t.hh = r & 1;                       // the two halves of a key tile run on neighbouring CTAs
+    r >>= 1;
+    t.b = r / p.Hkv;
+    t.hk = r % p.Hkv;
+    if (p.cu_q != nullptr) {
+        t.q_start = max(__ldg(p.cu_q + t.b), 0);
+        t.k_start = max(__ldg(p.cu_k + t.b), 0);
+        t.Lq = max(min(__ldg(p.cu_q + t.b + 1) - t.q_start, p.Tq - t.q_start), 0);
+        t.Lk = max(min(__ldg(p.cu_k + t.b + 1) - t.k_start, p.Tk - t.k_start), 0);
+    } else {
+        t.q_start = t.b * p.Sq;
+        t.Lq = p.Sq;
+        t.k_start = t.b * p.Sk;
+        t.Lk = p.Sk;
+    }
+    t.n0 = n * 128;
+    t.skip = t.n0 >= t.Lk;
+    int m_start = 0;
+    if (p.causal) {
+        const int first_row = t.n0 - (t.Lk - t.Lq);
+        m_start = first_row > 0 ? first_row / 64 : 0;
+    }
+    const int m_end = (t.Lq + 63) / 64;
+    t.m_start = m_start;
+    t.n_m = m_end > m_start ? m_end - m_start : 0;
+    t.n_it = t.n_m * p.group;
+    return t;
+}
+
+struct Cfg {
+    static constexpr uint32_t KV_BYTES = 128 * D * 2;    // 64 KB, four [128 x 64] boxes
+    static constexpr uint32_t QT_BYTES = 64 * D * 2;     // 32 KB, four [64 x 64] boxes
+    static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_Q = 2 * KV_BYTES, OFF_DO = OFF_Q + QT_BYTES,
+                              OFF_DS = OFF_DO + QT_BYTES,               // dS^T [128 keys][64 queries], 16 KB
+                              OFF_STAT = OFF_DS + 128 * 128, OFF_BAR = OFF_STAT + 2 * 64 * 4;
+    static constexpr int NUM_BARS = 9;
+    static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
+    static constexpr int THREADS = 384, LAUNCH_REGS = 168, COMPUTE_REGS = 232, OTHER_REGS = 136;
+    static_assert(128 * COMPUTE_REGS + 2 * 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
+};
+
+__global__ void __launch_bounds__(384, 1)
+    bwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ B256Params p) {
+    using C = Cfg;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);   // [64]
+    float* sDel = sLSE + 64;                                      // [64]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t b0 = smem_u32(bars);
+    const uint32_t kv_full = b0, kv_empty = b0 + 8, q_full = b0 + 16, q_empty = b0 + 24, s_full = b0 + 32,
+                   p_full = b0 + 40, dq_full = b0 + 48, dq_empty = b0 + 56, dkv_full = b0 + 64;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int PRODUCER = 8, MMA = 9;
+
+    if ((smem_u32(smem) & 1023u) != 0) {
+        if (threadIdx.x == 0) atomicCAS(p.status, 0, 2);
+        return;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bars + 0, 1);
+        mbar_init(bars + 1, 1);
+        mbar_init(bars + 2, 33);     // q_full: 32 producer lanes (statistics) + the TMA expect-tx arrival
+        mbar_init(bars + 3, 1);
+        mbar_init(bars + 4, 1);
+        mbar_init(bars + 5, 128);    // p_full
+        mbar_init(bars + 6, 1);
+        mbar_init(bars + 7, 128);    // dq_empty
+        mbar_init(bars + 8, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == PRODUCER && lane == 0) {
+        tma_prefetch_map(&tmQ);
+        tma_prefetch_map(&tmK);
+        tma_prefetch_map(&tmV);
+        tma_prefetch_map(&tmDO);
+    }
+    if (warp == MMA) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Watch w{abort_flag, p.status, p.timeout_ns};
+    const int G = p.group;
+
+    if (warp >= 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
+        if (warp == PRODUCER) {
+            uint32_t unit_it = 0, q_it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const U256 t = decode_u256(p, u);
+                if (t.skip || t.n_it == 0) continue;
+                if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(kv_full, 2 * C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
+                        tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
+                    }
+                }
+                ++unit_it;
+                for (int it = 0; it < t.n_it; ++it, ++q_it) {
+                    const int g = it / t.n_m;
+                    const int m0 = (t.m_start + it % t.n_m) * 64;
+                    const int h = t.hk * G + g;
+                    if (q_it > 0 && !mbar_wait(q_empty, (q_it - 1) & 1, w)) { ok = false; break; }
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int qi = lane * 2 + e;
+                        const int row = m0 + qi;
+                        const bool in = row < t.Lq;
+                        const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
+                        sLSE[qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
+                        sDel[qi] = in ? __ldg(p.delta + idx) : 0.f;
+                    }
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(q_full, 2 * C::QT_BYTES);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            tma_load_3d(smem_u32(smem + C::OFF_Q + c * 64 * 128), &tmQ, q_full, c * 64, h,
+                                        t.q_start + m0);
+                            tma_load_3d(smem_u32(smem + C::OFF_DO + c * 64 * 128), &tmDO, q_full, c * 64, h,
+                                        t.q_start + m0);
+                        }
+                    }
+                    mbar_arrive(q_full);
+                }
+            }
+            __syncwarp();
+        } else if (warp == MMA) {
+            if (lane == 0) {
+                constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);     // S^T, dP^T
+                constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, true);     // dV, dK halves
+                constexpr uint32_t id_q = idesc_bf16_f32(128, 64, true, true);       // dQ^T half
+                uint32_t unit_it = 0, q_it = 0;
+                bool ok = true;
+                for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                    const U256 t = decode_u256(p, u);
+                    if (t.skip || t.n_it == 0) continue;
+                    if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
+                    for (int it = 0; it < t.n_it; ++it, ++q_it) {
+                        if (!mbar_wait(q_full, q_it & 1, w)) { ok = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t ok_ = (kk >> 2) * 128 * 128 + (kk & 3) * 32;   // [128 x 64] boxes
+                            const uint32_t oq = (kk >> 2) * 64 * 128 + (kk & 3) * 32;      // [64 x 64] boxes
+                            umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + ok_), 16, 1024),
+                                    sdesc_sw128(smem_u32(smem + C::OFF_Q + oq), 16, 1024), id_s, kk > 0);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t ok_ = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+                            const uint32_t oq = (kk >> 2) * 64 * 128 + (kk & 3) * 32;
+                            umma_ss(tmem + C::COL_DP, sdesc_sw128(smem_u32(smem + C::OFF_V + ok_), 16, 1024),
+                                    sdesc_sw128(smem_u32(smem + C::OFF_DO + oq), 16, 1024), id_s, kk > 0);
+                        }
+                        umma_commit(s_full);
+                        if (!mbar_wait(p_full, q_it & 1, w)) { ok = false; break; }
+                        if (q_it > 0 && !mbar_wait(dq_empty, (q_it - 1) & 1, w)) { ok = false; break; }
+                        tc_fence_after();
+                        // dQ^T half = K[:, half]^T dS^T (K-dim = 128 keys)
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            umma_ss(tmem + C::COL_DQ,
+                                    sdesc_sw128(smem_u32(smem + C::OFF_K + 2 * t.hh * 128 * 128 + kk * 16 * 128),
+                                                128 * 128, 1024),
+                                    sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024), id_q,
+                                    kk > 0);
+                        }
+                        umma_commit(dq_full);
+                        // dV half += P^T dO[:, half], dK half += dS^T Q[:, half] (K-dim = 64 queries)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                            umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8,
+                                    sdesc_sw128(smem_u32(smem + C::OFF_DO + 2 * t.hh * 64 * 128 + kk * 16 * 128),
+                                                64 * 128, 1024),
+                                    id_g, acc);
+                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8,
+                                    sdesc_sw128(smem_u32(smem + C::OFF_Q + 2 * t.hh * 64 * 128 + kk * 16 * 128),
+                                                64 * 128, 1024),
+                                    id_g, acc);
+                        }
+                        umma_commit(q_empty);
+                    }
+                    if (!ok) break;
+                    umma_commit(dkv_full);
+                    umma_commit(kv_empty);
+                    ++unit_it;
+                }
+            }
+            __syncwarp();
+        } else if (warp < 8) {
+            // -------------------------------------------------------- dQ warpgroup (thread = head-dim row)
+            const int wq = warp - 4;
+            const int r = wq * 32 + lane;
+            const uint32_t lb = tmem_lane_base(wq);
+            uint32_t q_it = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                const U256 t = decode_u256(p, u);
+                if (t.skip || t.n_it == 0) continue;
+                for (int it = 0; it < t.n_it; ++it, ++q_it) {
+                    const int g = it / t.n_m;
+                    const int m0 = (t.m_start + it % t.n_m) * 64;
+                    const int h = t.hk * G + g;
+                    if (!mbar_wait(dq_full, q_it & 1, w)) { ok = false; break; }
+                    tc_fence_after();
+                    float* acc = p.dq_acc + (static_cast<size_t>(h) * p.Tq + t.q_start + m0) * D + t.hh * 128 + r;
+#pragma unroll 1
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t ra[32];
+                        tmem_ld32(tmem + lb + C::COL_DQ + cc * 32, ra);
+                        tmem_ld_wait_tie(ra);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int qc = cc * 32 + e;
+                            if (m0 + qc < t.Lq) atomicAdd(acc + static_cast<size_t>(qc) * D, __uint_as_float(ra[e]));
+                        }
+                    }
+                    tc_fence_before();
+                    mbar_arrive(dq_empty);
+                }
+            }
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
+        // ------------------------------------------------------------ compute warpgroup (thread = key row)
+        const int r = warp * 32 + lane;
+        const uint32_t lb = tmem_lane_base(warp);
+        const float c2 = p.scale_log2;
+        uint32_t unit_it = 0, q_it = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            const U256 t = decode_u256(p, u);
+            if (t.skip) continue;
+            const int kj = t.n0 + r;
+            const bool kvalid = kj < t.Lk;
+            const size_t krow = (static_cast<size_t>(t.k_start) + kj) * p.Hkv + t.hk;
+            if (t.n_it == 0) {
+                if (kvalid) {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < 16; ++c) {
+                        reinterpret_cast<uint4*>(p.dk + krow * D + t.hh * 128)[c] = z;
+                        reinterpret_cast<uint4*>(p.dv + krow * D + t.hh * 128)[c] = z;
+                    }
+                }
+                continue;
+            }
+            const int off = t.Lk - t.Lq;
+            for (int it = 0; it < t.n_it; ++it, ++q_it) {
+                const int m0 = (t.m_start + it % t.n_m) * 64;
+                if (!mbar_wait(s_full, q_it & 1, w)) { ok = false; break; }
+                if (!mbar_wait(q_full, q_it & 1, w)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sa[2][32], da[2][32];
+                tmem_ld32(tmem + lb + C::COL_S, sa[0]);
+                tmem_ld32(tmem + lb + C::COL_S + 32, sa[1]);
+                tmem_ld32(tmem + lb + C::COL_DP, da[0]);
+                tmem_ld32(tmem + lb + C::COL_DP + 32, da[1]);
+                tmem_ld_wait_tie(sa[0]);
+                reg_tie(sa[1]);
+                reg_tie(da[0]);
+                reg_tie(da[1]);
+                const int qmin = p.causal ? kj - off - m0 : -0x40000000;
+                const bool any_mask = __any_sync(0xffffffffu, !(kvalid && qmin <= 0));
+                const float2 c2v = make_float2(c2, c2);
+                uint8_t* ds_row = smem + C::OFF_DS + r * 128;
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t pp[16], dd[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int qc = half * 32 + e;
+                        const float2 sv = make_float2(__uint_as_float(sa[half][e]), __uint_as_float(sa[half][e + 1]));
+                        const float2 dv = make_float2(__uint_as_float(da[half][e]), __uint_as_float(da[half][e + 1]));
+                        const float2 a = ffma2(sv, c2v, make_float2(-sLSE[qc], -sLSE[qc + 1]));
+                        float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                        if (any_mask) {
+                            pr.x = (kvalid && qc >= qmin) ? pr.x : 0.f;
+                            pr.y = (kvalid && qc + 1 >= qmin) ? pr.y : 0.f;
+                        }
+                        const float2 ds = fmul2(pr, fadd2(dv, make_float2(-sDel[qc], -sDel[qc + 1])));
+                        pp[e / 2] = pack_bf16x2(pr.x, pr.y);
+                        dd[e / 2] = pack_bf16x2(ds.x, ds.y);
+                    }
+                    tmem_st16(tmem + lb + C::COL_S + 16 * half, pp);
+                    tmem_st16(tmem + lb + C::COL_DP + 16 * half, dd);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int cin = half * 4 + q4;
+                        *reinterpret_cast<uint4*>(ds_row + ((cin ^ (r & 7)) << 4)) =
+                            make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
+                    }
+                }
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(p_full);
+            }
+            if (!ok) break;
+            if (!mbar_wait(dkv_full, unit_it & 1, w)) { ok = false; break; }
+            ++unit_it;
+            tc_fence_after();
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col = which == 0 ? C::COL_DV : C::COL_DK;
+                const float2 mul2 = which == 0 ? make_float2(1.f, 1.f) : make_float2(p.scale, p.scale);
+                __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + krow * D + t.hh * 128;
+#pragma unroll 1
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint32_t ra[32];
+                    tmem_ld32(tmem + lb + col + cc * 32, ra);
+                    tmem_ld_wait_tie(ra);
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 v =
+                            fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), mul2);
+                        pk[e] = pack_bf16x2(v.x, v.y);
+                    }
+                    if (kvalid) {
+                        uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
+                }
+            }
+            tc_fence_before();
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) {
+        }
+    }
+    if (warp == MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// dQ[tok][h][:] = bf16(scale * dQacc[h][tok][:])
+__global__ void __launch_bounds__(256) bwd256_convert_kernel(const float* dq_acc, __nv_bfloat16* dq, int Tq, int Hq,
+                                                             float scale) {
+    const long long n2 = static_cast<long long>(Tq) * Hq * (D / 2);
+    for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n2;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+        const long long e = 2 * i;
+        const int d = static_cast<int>(e % D);
+        const long long th = e / D;               // tok * Hq + h
+        const int h = static_cast<int>(th % Hq);
+        const long long tok = th / Hq;
+        const float2 v = *reinterpret_cast<const float2*>(dq_acc + (static_cast<size_t>(h) * Tq + tok) * D + d);
+        reinterpret_cast<uint32_t*>(dq)[i] = pack_bf16x2(v.x * scale, v.y * scale);
+    }
+}
+
+}  // namespace
+
+int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,
+                       void* dq, void* dk, void* dv, const Device& dev, cudaStream_t stream) {
+    using C = Cfg;
+    alignas(64) CUtensorMap mq, mk, mv, mdo;
+    const uint64_t rq = static_cast<uint64_t>(pr.Hq) * D * 2, rk = static_cast<uint64_t>(pr.Hkv) * D * 2;
+    if (!make_map_3d_bf16(&mq, pr.q, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, 64)) return 5;
+    if (!make_map_3d_bf16(&mdo, dout, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, 64)) return 5;
+    if (!make_map_3d_bf16(&mk, pr.k, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+    if (!make_map_3d_bf16(&mv, pr.v, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+    B256Params p;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.dq_acc = dq_acc;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.cu_q = pr.cu_q;
+    p.cu_k = pr.cu_k;
+    p.num_seqs = pr.num_seqs;
+    p.Sq = pr.Sq;
+    p.Sk = pr.Sk;
+    p.Tq = pr.Tq;
+    p.Tk = pr.Tk;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.group = pr.Hq / pr.Hkv;
+    const long long units = static_cast<long long>((pr.Sk + 127) / 128) * pr.num_seqs * pr.Hkv * 2;
+    if (units > 0x7fffffffLL) return 2;
+    p.num_units = static_cast<int>(units);
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale * 1.4426950408889634f;
+    p.causal = pr.causal;
+    p.timeout_ns = dev.timeout_ns;
+    p.status = dev.status;
+    static bool set[64] = {};
+    if (!set[dev.id & 63]) {
+        if (cudaFuncSetAttribute(bwd256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(C::SMEM)) != cudaSuccess)
+            return 5;
+        cudaFuncAttributes fa_attr;
+        if (cudaFuncGetAttributes(&fa_attr, bwd256_kernel) != cudaSuccess || fa_attr.numRegs != C::LAUNCH_REGS)
+            return 2;
+        set[dev.id & 63] = true;
+    }
+    const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
+    if (grid > 0) {
+        prof_before(1, stream);
+        bwd256_kernel<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        prof_after(1, stream);
+        if (cudaPeekAtLastError() != cudaSuccess) return 5;
+    }
+    const long long n2 = static_cast<long long>(pr.Tq) * pr.Hq * (D / 2);
+    long long blocks = (n2 + 255) / 256;
+    if (blocks > static_cast<long long>(dev.num_sms) * 32) blocks = static_cast<long long>(dev.num_sms) * 32;
+    bwd256_convert_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), pr.Tq,
+                                                                        pr.Hq, pr.scale);
+    return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
+}
+
+}  // namespace fa

@@ -44,6 +44,9 @@ void prof_after(int kernel_id, cudaStream_t s);
 int launch_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream);
 
 size_t bwd_workspace_bytes(long long Tq, int Hq, int D);
+// head dim 256: main backward kernel + dQ convert (after the shared preprocess)
+int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,
+                       void* dq, void* dk, void* dv, const Device& dev, cudaStream_t stream);
 int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
                void* dv, void* workspace, const Device& dev, cudaStream_t stream);
 

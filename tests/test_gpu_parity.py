@@ -56,10 +56,10 @@ def test_dense_ragged_gqa(D, causal, Sq, Sk):
 
 
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("Sq,Sk", [(300, 300), (129, 257)])
-def test_dense_d256_forward(causal, Sq, Sk):
-    w = W.dense(1, Sq, Sk, 4, 1, 256, causal, seed=11, with_grad=False)
-    H.check_dense(w, backward=False)
+@pytest.mark.parametrize("Sq,Sk", [(300, 300), (129, 257), (200, 70)])
+def test_dense_d256(causal, Sq, Sk):
+    w = W.dense(1, Sq, Sk, 4, 1, 256, causal, seed=11)
+    H.check_dense(w)
 
 
 def test_mqa_and_wide_group():
@@ -114,10 +114,10 @@ def test_varlen_unequal_q_and_k_lengths():
     H.check_varlen(w)
 
 
-def test_varlen_d256_forward():
+def test_varlen_d256():
     lens = [1, 200, 129, 64]
-    w = W.varlen(lens, lens, 4, 4, 256, True, seed=6, with_grad=False)
-    H.check_varlen(w, backward=False)
+    w = W.varlen(lens, lens, 4, 2, 256, True, seed=6)
+    H.check_varlen(w)
 
 
 def test_varlen_matches_dense_layout():
