@@ -184,7 +184,8 @@ __global__ void __launch_bounds__(512, 1)
             // -------------------------------------------------------- producer (whole warp)
             uint32_t unit_it = 0, q_it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+                if (u >= p.num_units) continue;
                 const BUnit t = decode_bunit(p, u);
                 if (t.skip || t.n_it == 0) continue;
                 if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
@@ -237,7 +238,8 @@ __global__ void __launch_bounds__(512, 1)
                 constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);      // dQ, 64 columns at a time
                 uint32_t unit_it = 0, q_it = 0, g_it = 0;
                 bool ok = true;
-                for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+                for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+                    if (u >= p.num_units) continue;
                     const BUnit t = decode_bunit(p, u);
                     if (t.skip || t.n_it == 0) continue;
                     if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
@@ -302,7 +304,8 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t lb = tmem_lane_base(wq);
         uint32_t g_it = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+            if (u >= p.num_units) continue;
             const BUnit t = decode_bunit(p, u);
             if (t.skip || t.n_it == 0) continue;
             for (int it = 0; it < t.n_it; ++it, ++g_it) {
@@ -340,7 +343,8 @@ __global__ void __launch_bounds__(512, 1)
         const float c2 = p.scale_log2;
         uint32_t unit_it = 0, q_it = 0, g_it = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+            if (u >= p.num_units) continue;
             const BUnit t = decode_bunit(p, u);
             if (t.skip) continue;
             const int kj = t.n0 + r;                 // key index inside the sequence

@@ -20,9 +20,10 @@
 //     O_i += P_i V (P from tensor memory, V N-major in shared memory).
 //   Order per KV tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the tensor
 //   core computes one tile's scores while the other tile's softmax runs.
-//   * work units (sequence, head, block of NQ*128 query rows) are taken
-//     round-robin in heaviest-first order (query blocks with most KV tiles first
-//     for causal masks); causal blocks stop at the last KV tile they can see.
+//   * work units (sequence, head, block of NQ*128 query rows) are listed
+//     heaviest first (query blocks with most KV tiles first for causal masks)
+//     and dealt to the persistent CTAs in boustrophedon order (snake_unit);
+//     causal blocks stop at the last KV tile they can see.
 //
 // Exactness of the deferred rescale: P, l and O are all taken against the same
 // reference value m_ref of the row, which is only raised when a tile's max
@@ -183,7 +184,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     if (warp == PRODUCER) {
         if (lane == 0) {
             uint32_t kv_it = 0, q_it = 0;
-            for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0; u = snake_unit(++k, p.num_units)) {
+                if (u >= p.num_units) continue;
                 const Unit t = decode_unit<ROWS, BK>(p, u);
                 if (t.skip || t.n_kv == 0) continue;
                 const int hk = t.h / p.group;
@@ -242,7 +244,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             };
             uint32_t kv_it = 0, q_it = 0, p_it = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+                if (u >= p.num_units) continue;
                 const Unit t = decode_unit<ROWS, BK>(p, u);
                 if (t.skip || t.n_kv == 0) continue;
                 for (int i = 0; i < NQ && ok; ++i)
@@ -309,7 +312,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
         const float c2 = p.scale_log2;
         uint32_t s_it = 0, pv_total = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < p.num_units && ok; u += gridDim.x) {
+        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+            if (u >= p.num_units) continue;
             const Unit t = decode_unit<ROWS, BK>(p, u);
             if (t.skip) continue;
             const int row = t.q0 + i * BM + r;

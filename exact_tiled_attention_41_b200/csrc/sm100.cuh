@@ -294,4 +294,16 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
+// Persistent schedule over work units sorted heaviest first: round k of CTA c takes unit
+// k*G + c on even rounds and k*G + (G-1-c) on odd rounds (a boustrophedon), so the CTA that
+// got the heaviest unit of one round gets the lightest of the next.  Returns -1 past the end
+// of the list (stop) and num_units (skip) when this round's slot is empty.
+__device__ __forceinline__ int snake_unit(int k, int num_units) {
+    const int G = static_cast<int>(gridDim.x), c = static_cast<int>(blockIdx.x);
+    const long long base = static_cast<long long>(k) * G;
+    if (base >= num_units) return -1;
+    const long long u = base + ((k & 1) ? (G - 1 - c) : c);
+    return u < num_units ? static_cast<int>(u) : num_units;
+}
+
 }  // namespace fa
