@@ -21,7 +21,10 @@
 //                    memory (written back as bf16, dS^T also to shared memory);
 //                    dV (warpgroup 0) / dK (warpgroup 1) epilogue
 //        warps 8-11  dQ: thread = query row; reads the dQ tile from tensor memory
-//                    and adds it to the fp32 accumulator (vector atomics)
+//                    and adds it to the fp32 accumulator (vector atomics); each half
+//                    of the tile is released as soon as it is in registers, so the
+//                    next S^T (first half) and dP^T (second half) wait as little as
+//                    possible on the reduction traffic
 //        warp 12     producer: K, V once per unit; Q, dO tiles (TMA) and the
 //                    tile's LSE2 / Delta (plain loads) through a 2-stage ring
 //        warp 13     tensor memory and every tcgen05 MMA, in this order per tile:
@@ -104,7 +107,7 @@ struct BwdCfg {
     static constexpr uint32_t OFF_K = 0, OFF_V = T_BYTES, OFF_Q = 2 * T_BYTES, OFF_DO = (2 + ST) * T_BYTES,
                               OFF_DS = (2 + 2 * ST) * T_BYTES, OFF_STAT = OFF_DS + DS_BYTES,
                               OFF_BAR = OFF_STAT + 2 * ST * 128 * 4;
-    static constexpr int NUM_BARS = 2 + 2 * ST + 5;
+    static constexpr int NUM_BARS = 2 + 2 * ST + 6;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
     // tensor memory: dV | dK | S^T | dP^T.  After the gradient step P^T and dS^T (bf16) occupy the
     // low 64 columns of S^T and dP^T; dQ (fp32) is accumulated into their free high 64 columns.
@@ -137,7 +140,7 @@ __global__ void __launch_bounds__(512, 1)
     auto q_full = [&](int s) { return b0 + 8u * (2 + s); };
     auto q_empty = [&](int s) { return b0 + 8u * (2 + ST + s); };
     const uint32_t s_full = b0 + 8u * (2 + 2 * ST), p_full = s_full + 8, dq_full = s_full + 16,
-                   dq_empty = s_full + 24, dkv_full = s_full + 32;
+                   dq_empty = s_full + 24, dkv_full = s_full + 32, dq_empty_hi = s_full + 40;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PRODUCER = 12, MMA = 13;
@@ -156,8 +159,9 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bars + 2 + 2 * ST + 0, 1);    // s_full
         mbar_init(bars + 2 + 2 * ST + 1, 256);  // p_full: both compute warpgroups
         mbar_init(bars + 2 + 2 * ST + 2, 1);    // dq_full
-        mbar_init(bars + 2 + 2 * ST + 3, 128);  // dq_empty
+        mbar_init(bars + 2 + 2 * ST + 3, 128);  // dq_empty: dQ columns in the S^T region read out
         mbar_init(bars + 2 + 2 * ST + 4, 1);    // dkv_full
+        mbar_init(bars + 2 + 2 * ST + 5, 128);  // dq_empty_hi: dQ columns in the dP^T region read out
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -256,6 +260,9 @@ __global__ void __launch_bounds__(512, 1)
                             umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + o), 16, 1024),
                                     sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
                         }
+                        // the previous tile's dQ columns in the dP^T region must be read out first
+                        if (g_it > 0 && !mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
+                        tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
@@ -322,6 +329,13 @@ __global__ void __launch_bounds__(512, 1)
                     uint32_t ra[32];
                     tmem_ld32(tmem + lb + C::COL_DQ(cc >> 1) + (cc & 1) * 32, ra);
                     tmem_ld_wait_tie(ra);
+                    // release each half of the tile as soon as it sits in registers: the next S^T
+                    // overwrites the first half, the next dP^T the second
+                    if (cc == 1 || cc == D / 32 - 1) {
+                        tc_fence_before();
+                        if (cc == 1) mbar_arrive(dq_empty);
+                        if (cc == D / 32 - 1) mbar_arrive(dq_empty_hi);
+                    }
                     if (valid) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
@@ -330,8 +344,6 @@ __global__ void __launch_bounds__(512, 1)
                                                   __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3])));
                     }
                 }
-                tc_fence_before();
-                mbar_arrive(dq_empty);
             }
         }
     } else {
