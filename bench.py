@@ -42,6 +42,22 @@ def fwd_flops(B, H, Sq, Sk, D, causal):
     return 4.0 * B * H * Sq * Sk * D * (0.5 if causal else 1.0)
 
 
+def max_over_ranks(value, world, device="cpu"):
+    """The slowest rank's figure; every rank takes part in the same collective (no-op for one rank)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tflops(step_flops, world, ms_per_step):
+    """Whole-job throughput of `world` replicas that each did one step in (at most) ms_per_step."""
+    return world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -254,14 +270,11 @@ def run_ours(args, rank, world, local_rank):
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     _, n_f, ms_f = abi.fa_profile_read(abi.FA_KERNEL_FWD)
     _, n_b, ms_b = abi.fa_profile_read(abi.FA_KERNEL_BWD)
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
     if abi.fa_get_device_status() != 0:
         raise RuntimeError("a kernel reported a device-side timeout during the timed region")
     ms_per_step = total_ms / args.steps
-    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    value = aggregate_tflops(step_flops, world, ms_per_step)
 
     # ----------------------------------------------------------------- end to end through the public API
     e2e_steps = min(args.steps, 30)
@@ -289,12 +302,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
-    e2e_value = world * step_flops / (e2e_ms * 1e-3) / 1e12
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
+    e2e_value = aggregate_tflops(step_flops, world, e2e_ms)
 
     extras = {}
     if world == 1 and not args.no_extras:
