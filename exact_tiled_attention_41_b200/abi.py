@@ -30,7 +30,7 @@ EXPORTS = (
     "fa_fwd_kvcache", "fa_fwd_kvcache_workspace_size", "fa_status_string", "fa_get_device_status",
     "fa_set_wait_timeout_ns", "fa_debug_wait_timeout_selftest", "fa_debug_umma_selftest",
     "fa_profile_begin", "fa_profile_read",
-    "fa_fwd_kvcache_noalloc", "fa_fwd_kvcache_noalloc_scratch_bytes",
+    "fa_fwd_kvcache_noalloc", "fa_fwd_kvcache_noalloc_scratch_bytes", "fa_debug_exp2_selftest",
 )
 
 FA_KERNEL_FWD = 0
@@ -63,6 +63,7 @@ _SIGS = {
     "fa_profile_read": (_I, [_I, ctypes.POINTER(_I), ctypes.POINTER(_F)]),
     "fa_fwd_kvcache_noalloc": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P]),
     "fa_fwd_kvcache_noalloc_scratch_bytes": (_Z, []),
+    "fa_debug_exp2_selftest": (_I, [_P, _P, _I, _P]),
 }
 
 _lib = None
@@ -181,6 +182,10 @@ def fa_debug_wait_timeout_selftest(timeout_ns: int, stream=None) -> int:
 
 def fa_debug_umma_selftest(a, b, c, mode: int, stream=None) -> int:
     return load().fa_debug_umma_selftest(_ptr(a), _ptr(b), _ptr(c), int(mode), _stream(stream))
+
+
+def fa_debug_exp2_selftest(x, y, n: int, stream=None) -> int:
+    return load().fa_debug_exp2_selftest(_ptr(x), _ptr(y), int(n), _stream(stream))
 
 
 def fa_profile_begin(enable: int) -> int:

@@ -357,6 +357,12 @@ int fa_debug_wait_timeout_selftest(unsigned long long timeout_ns, fa_stream_t st
     return launch_wait_selftest(timeout_ns, dev, static_cast<cudaStream_t>(stream));
 }
 
+int fa_debug_exp2_selftest(const float* x, float* y, int n, fa_stream_t stream) {
+    if (!x || !y || n <= 0 || (n & 1)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(y)) return FA_ERR_ALIGNMENT;
+    return launch_exp2_selftest(x, y, n, static_cast<cudaStream_t>(stream)) == 0 ? FA_OK : FA_ERR_CUDA;
+}
+
 int fa_debug_umma_selftest(const void* a, const void* b, float* c, int mode, fa_stream_t stream) {
     if (!a || !b || !c || mode < 0 || mode > 2) return FA_ERR_INVALID_ARG;
     if (!aligned16(a) || !aligned16(b) || !aligned16(c)) return FA_ERR_ALIGNMENT;

@@ -116,6 +116,11 @@ struct FwdCfg {
 };
 
 constexpr float kDeferLog2 = 8.0f;
+// Share of the softmax exponentials computed on the FMA pipe (exp2_fma2) instead of the
+// multi-function unit, whose 16 results per clock per SM match the tensor rate at D = 128:
+// one pair in kFmaExpEvery, 0 = none.  Measured on B200: moving a quarter of them made the
+// forward slower (the softmax is bound by latency and issue, not by the exp2 unit), so it is off.
+constexpr int kFmaExpEvery = 0;
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int D, int NQ, int BK, int KST>
@@ -399,7 +404,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     for (int e = 0; e < 32; ++e) {
                         // exp(scale * s - scale * m) as exp2 of one fused multiply-add per pair
                         const float2 x = ffma2(make_float2(s[half * 64 + 2 * e], s[half * 64 + 2 * e + 1]), c2v, nms);
-                        const float2 p2 = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+                        // one pair in kFmaExpEvery goes to the FMA pipe, the rest to the exp2 unit
+                        const float2 p2 = (kFmaExpEvery > 0 && e % kFmaExpEvery == kFmaExpEvery - 1)
+                                              ? exp2_fma2(x)
+                                              : make_float2(ex2_approx(x.x), ex2_approx(x.y));
                         if (e & 1) sum1 = fadd2(sum1, p2); else sum0 = fadd2(sum0, p2);
                         pk[e] = pack_bf16x2(p2.x, p2.y);
                     }

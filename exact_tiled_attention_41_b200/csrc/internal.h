@@ -70,6 +70,7 @@ size_t decode_workspace_bytes(int B, int Hq, int Hkv, int cap, int D, int chunk)
 int launch_decode(const Decode& d, const Device& dev, cudaStream_t stream);
 
 int launch_wait_selftest(unsigned long long timeout_ns, const Device& dev, cudaStream_t stream);
+int launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream);
 int launch_umma_selftest(const void* a, const void* b, float* c, int mode, const Device& dev, cudaStream_t stream);
 
 // cuTensorMapEncodeTiled, fetched through the runtime so the library needs no -lcuda.

@@ -23,6 +23,22 @@ __global__ void wait_selftest_kernel(unsigned long long limit_ns, int* status) {
     (void)mbar_wait(smem_u32(&bar), 0, w);
 }
 
+// y = 2^x through the FMA-pipe exponential used by the softmax kernels (pairs of elements).
+__global__ void exp2_selftest_kernel(const float* x, float* y, int n2) {
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n2; i += gridDim.x * blockDim.x) {
+        const float2 r = exp2_fma2(make_float2(x[2 * i], x[2 * i + 1]));
+        y[2 * i] = r.x;
+        y[2 * i + 1] = r.y;
+    }
+}
+
+int launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream) {
+    if (n <= 0 || (n & 1)) return 1;
+    const int n2 = n / 2;
+    exp2_selftest_kernel<<<(n2 + 255) / 256 < 1024 ? (n2 + 255) / 256 : 1024, 256, 0, stream>>>(x, y, n2);
+    return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
+}
+
 int launch_wait_selftest(unsigned long long timeout_ns, const Device& dev, cudaStream_t stream) {
     if (timeout_ns == 0 || timeout_ns > 10000000000ull) return 1;
     wait_selftest_kernel<<<1, 32, 0, stream>>>(timeout_ns, dev.status);

@@ -287,6 +287,30 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
     return r;
 }
 
+// Two exp2 on the FMA pipe, for the share of the softmax exponentials taken off the
+// multi-function unit.  x = j + f with j = rint(x) (rounding by adding and subtracting
+// 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f is a degree-6 polynomial whose coefficients minimise the
+// maximum relative error on [-1/2, 1/2] (Remez exchange, csrc/fit_exp2_poly.py): worst relative
+// error 1.0e-7 in fp32 over [-126, 8], about 2 ulp, like the hardware ex2.approx.  2^j is applied
+// by adding j to the exponent field (the shift drops the bias bits of the rounding constant).
+// Arguments below -125 (including -inf) give exactly 0 (results under 2^-125 are dropped, as
+// ex2.approx.ftz drops those under 2^-126; the exponent add stays in the normal range); x <= 127.
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+    const float2 t = fadd2(x, make_float2(kRound, kRound));
+    const float2 nj = fadd2(make_float2(kRound, kRound), make_float2(-t.x, -t.y));   // -rint(x)
+    const float2 f = fadd2(x, nj);
+    float2 p = ffma2(make_float2(1.5345812e-4f, 1.5345812e-4f), f, make_float2(1.3399931e-3f, 1.3399931e-3f));
+    p = ffma2(p, f, make_float2(9.618489e-3f, 9.618489e-3f));
+    p = ffma2(p, f, make_float2(5.5503286e-2f, 5.5503286e-2f));
+    p = ffma2(p, f, make_float2(2.4022646e-1f, 2.4022646e-1f));
+    p = ffma2(p, f, make_float2(6.931472e-1f, 6.931472e-1f));
+    p = ffma2(p, f, make_float2(1.0f, 1.0f));
+    const uint32_t bx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
+    const uint32_t by = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
+    return make_float2(x.x < -125.f ? 0.f : __uint_as_float(bx), x.y < -125.f ? 0.f : __uint_as_float(by));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);

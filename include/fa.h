@@ -230,6 +230,12 @@ FA_API int fa_debug_wait_timeout_selftest(unsigned long long timeout_ns, fa_stre
  */
 FA_API int fa_debug_umma_selftest(const void* a, const void* b, float* c, int mode, fa_stream_t stream);
 
+/* fa_debug_exp2_selftest: y[i] = 2^x[i] for n (even) device floats, computed with the
+ * FMA-pipe exponential the softmax kernels use for part of their exponentials, so that
+ * its accuracy can be checked against CUDA's exp2f.  Asynchronous on `stream`.
+ */
+FA_API int fa_debug_exp2_selftest(const float* x, float* y, int n, fa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -31,6 +31,30 @@ def test_tensor_core_selftest(mode):
     np.testing.assert_allclose(c.cpu().double().numpy(), ref, rtol=0, atol=1e-3)
 
 
+def test_fma_pipe_exp2_matches_cuda_exp2f():
+    # the softmax kernels take part of their exponentials off the multi-function unit; that
+    # polynomial must be as accurate as CUDA's own exp2f (about 2 ulp) over the range they use
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1 << 20), torch.rand(1 << 20) * 16 - 12,
+                   torch.tensor([0.0, 0.5, -0.5, 1.0, -1.0, 7.99, -124.9, -125.0, 8.0, 3.0])]).float()
+    x = x[: (x.numel() // 2) * 2].contiguous()
+    xd = x.cuda()
+    y = torch.empty_like(xd)
+    assert abi.fa_debug_exp2_selftest(xd, y, x.numel()) == 0
+    ref_cuda = torch.exp2(xd)                       # CUDA exp2f
+    torch.cuda.synchronize()
+    ref64 = torch.exp2(x.double())
+    rel = ((y.cpu().double() - ref64) / ref64).abs()
+    rel_cuda = ((ref_cuda.cpu().double() - ref64) / ref64).abs()
+    assert rel.max().item() <= 2.5e-7
+    assert rel.max().item() <= 2.5 * max(rel_cuda.max().item(), 6e-8)
+    # arguments below -125, and -inf (masked scores), give exactly zero
+    z = torch.tensor([-125.5, -126.0, -200.0, float("-inf")], dtype=torch.float32).cuda()
+    yz = torch.full_like(z, 1.0)
+    assert abi.fa_debug_exp2_selftest(z, yz, 4) == 0
+    torch.cuda.synchronize()
+    assert torch.all(yz == 0)
+
+
 def test_bounded_wait_reports_timeout_instead_of_hanging():
     assert abi.fa_get_device_status() == 0
     assert abi.fa_debug_wait_timeout_selftest(20_000_000) == 0      # 20 ms
