@@ -56,6 +56,7 @@ struct FwdParams {
 
 struct Unit {
     int b, h, q_start, k_start, Lq, Lk, q0, n_kv;
+    int n_tile[2];   // KV tiles seen by query tile 0 / 1 (0: the tile has no row inside the sequence)
     bool skip;
 };
 
@@ -85,12 +86,17 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     }
     t.q0 = m * ROWS;
     t.skip = t.q0 >= t.Lq;
-    int kend = t.Lk;
-    if (p.causal) {
-        const int last_row = min(t.q0 + ROWS, t.Lq) - 1;
-        kend = min(kend, last_row + (t.Lk - t.Lq) + 1);
+    t.n_kv = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int row_begin = t.q0 + 128 * i;              // query tiles are 128 rows
+        const int row_end = min(row_begin + 128, t.Lq);   // exclusive
+        int kend = row_end > row_begin ? t.Lk : 0;
+        if (p.causal && row_end > row_begin) kend = min(kend, row_end - 1 + (t.Lk - t.Lq) + 1);
+        t.n_tile[i] = kend > 0 ? (kend + BK - 1) / BK : 0;
+        if (i * 128 < ROWS) t.n_kv = max(t.n_kv, t.n_tile[i]);
+        else t.n_tile[i] = 0;
     }
-    t.n_kv = kend > 0 ? (kend + BK - 1) / BK : 0;
     return t;
 }
 
@@ -105,9 +111,9 @@ struct FwdCfg {
     // NQ softmax warpgroups + one warpgroup holding the producer warp, the MMA warp and two idle warps
     static constexpr int THREADS = (4 * NQ + 4) * 32;
     // register split with setmaxnreg (NQ = 2): launch at 168 per thread (384 x 168 = 64512),
-    // the producer/MMA warpgroup drops to 72 and the two softmax warpgroups rise to 216:
-    // 2 x 128 x 216 + 128 x 72 = 64512.  The host checks the launch count before the first launch.
-    static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 216, OTHER_REGS = 72;
+    // the producer/MMA warpgroup drops to 96 and the two softmax warpgroups rise to 200:
+    // 2 x 128 x 200 + 128 x 96 = 63488 <= 64512.  The host checks the launch count before the first launch.
+    static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 200, OTHER_REGS = 96;
     static_assert(NQ != 2 || 2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
     static constexpr uint32_t S_COL(int i) { return i * BK; }
     static constexpr uint32_t O_COL(int i) { return NQ * BK + i * D; }
@@ -247,7 +253,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                             idesc_pv, (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            uint32_t kv_it = 0, q_it = 0, p_it = 0;
+            uint32_t kv_it = 0, q_it = 0, p_it[NQ] = {};
             bool ok = true;
             for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
                 if (u >= p.num_units) continue;
@@ -262,6 +268,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     if (!mbar_wait(k_full(st), (kv_it / KST) & 1, w)) break;
                     tc_fence_after();
                     for (int i = 0; i < NQ; ++i) {
+                        if (t.n_tile[i] == 0) continue;
                         issue_qk(i, st);
                         umma_commit(s_full(i));
                     }
@@ -269,32 +276,36 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     if (t.n_kv == 1)
                         for (int i = 0; i < NQ; ++i) umma_commit(q_empty(i));
                 }
+                // query tile i stops after its own last visible KV tile (n_tile[i] <= n_kv)
                 for (int j = 0; j < t.n_kv && ok; ++j) {
                     const uint32_t cur = kv_it + j;
                     const int st = cur % KST;
                     const uint32_t nxt = cur + 1;
                     const int stn = nxt % KST;
-                    const bool has_next = j + 1 < t.n_kv;
                     if (!mbar_wait(v_full(st), (cur / KST) & 1, w)) { ok = false; break; }
                     tc_fence_after();
+                    bool k_ready = false;
                     for (int i = 0; i < NQ; ++i) {
-                        if (!mbar_wait(p_full(i), p_it & 1, w)) { ok = false; break; }
-                        tc_fence_after();
-                        issue_pv(i, st, j > 0);
-                        umma_commit(o_full(i));
-                        if (has_next) {
-                            if (i == 0) {
+                        if (j < t.n_tile[i]) {
+                            if (!mbar_wait(p_full(i), p_it[i] & 1, w)) { ok = false; break; }
+                            ++p_it[i];
+                            tc_fence_after();
+                            issue_pv(i, st, j > 0);
+                            umma_commit(o_full(i));
+                        }
+                        if (j + 1 < t.n_tile[i]) {
+                            if (!k_ready) {
                                 if (!mbar_wait(k_full(stn), (nxt / KST) & 1, w)) { ok = false; break; }
                                 tc_fence_after();
+                                k_ready = true;
                             }
                             issue_qk(i, stn);
                             umma_commit(s_full(i));
                         }
                     }
                     if (!ok) break;
-                    ++p_it;
                     umma_commit(v_empty(st));
-                    if (has_next) {
+                    if (j + 1 < t.n_kv) {
                         umma_commit(k_empty(stn));
                         if (j + 2 == t.n_kv)
                             for (int i = 0; i < NQ; ++i) umma_commit(q_empty(i));
@@ -325,7 +336,8 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             const bool valid = row < t.Lq;
             __nv_bfloat16* orow = p.o + (static_cast<size_t>(t.q_start + row) * p.Hq + t.h) * D;
             float* lse_ptr = p.lse + t.b * p.lse_sB + t.h * p.lse_sH + static_cast<long long>(t.q_start) * p.lse_sT + row;
-            if (t.n_kv == 0) {
+            const int n_mine = t.n_tile[i];          // KV tiles this query tile sees
+            if (n_mine == 0) {
                 if (valid) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
                     for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(orow)[c] = z;
@@ -337,7 +349,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             const int key_lim = p.causal ? min(t.Lk - 1, row + off) : (t.Lk - 1);
             float m_ref = -INFINITY;
             float l = 0.f;
-            for (int j = 0; j < t.n_kv; ++j) {
+            for (int j = 0; j < n_mine; ++j) {
                 if (!mbar_wait(s_full(i), s_it & 1, w)) { ok = false; break; }
                 ++s_it;
                 tc_fence_after();
@@ -422,7 +434,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                 mbar_arrive(p_full(i));
             }
             if (!ok) break;
-            pv_total += t.n_kv;
+            pv_total += n_mine;
             // ------------------------------------------------ epilogue: O / l, LSE
             if (!mbar_wait(o_full(i), (pv_total - 1) & 1, w)) { ok = false; break; }
             tc_fence_after();
