@@ -508,28 +508,35 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
              i += static_cast<long long>(gridDim.x) * blockDim.x)
             z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    for (long long row = gw; row < rows; row += (static_cast<long long>(gridDim.x) * blockDim.x) >> 5) {
-        const int tok = static_cast<int>(row / Hq), h = static_cast<int>(row % Hq);
-        constexpr int PER = D / 32;
-        const __nv_bfloat16* o = out + row * D + lane * PER;
-        const __nv_bfloat16* g = dout + row * D + lane * PER;
+    // D/8 lanes per row, 16 bytes of O and of dO per lane; 32/(D/8) rows per warp per pass
+    constexpr int LPR = D / 8, RPW = 32 / LPR;
+    const int sub = lane / LPR, sl = lane % LPR;
+    const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    for (long long row0 = gw * RPW; row0 < rows; row0 += nwarps * RPW) {
+        const long long row = row0 + sub;
         float s = 0.f;
+        if (row < rows) {
+            const uint4 a = *reinterpret_cast<const uint4*>(out + row * D + sl * 8);
+            const uint4 b = *reinterpret_cast<const uint4*>(dout + row * D + sl * 8);
+            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-        for (int e = 0; e < PER; e += 2) {
-            const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + e);
-            const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(g + e);
-            s = fmaf(__bfloat162float(a.x), __bfloat162float(b.x), s);
-            s = fmaf(__bfloat162float(a.y), __bfloat162float(b.y), s);
+            for (int e = 0; e < 4; ++e) {
+                const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
+                const float2 fb = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bv[e]));
+                s = fmaf(fa.x, fb.x, s);
+                s = fmaf(fa.y, fb.y, s);
+            }
         }
 #pragma unroll
-        for (int x = 16; x > 0; x >>= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
-        if (lane == 0) {
+        for (int x = LPR / 2; x > 0; x >>= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
+        if (sl == 0 && row < rows) {
+            const int tok = static_cast<int>(row / Hq), h = static_cast<int>(row % Hq);
             long long li;
             if (lse_sT) {
                 li = h * lse_sH + tok;
             } else {
-                const int b = tok / Sq, i = tok - b * Sq;
-                li = b * lse_sB + h * lse_sH + i;
+                const int bb = tok / Sq, i = tok - bb * Sq;
+                li = bb * lse_sB + h * lse_sH + i;
             }
             const float l = lse[li];
             const size_t wi = static_cast<size_t>(h) * Tq + tok;
