@@ -16,6 +16,11 @@ Sources (page titles as published; section named in brackets):
   entry 2.1: the causal mask is aligned to the bottom-right corner of the
   attention matrix (key j is kept for query i iff j <= i + seqlen_k - seqlen_q);
   a query row whose mask is all zero produces an output of zero.
+* flash-attention README, ``flash_attn_func`` docstring (sliding window local
+  attention, changelog 2.3): with window_size = (left, right) other than
+  (-1, -1), query i attends only to the keys j with
+  i + seqlen_k - seqlen_q - left <= j <= i + seqlen_k - seqlen_q + right;
+  -1 means that side of the window is unbounded.
 * flash-attention README, ``flash_attn_with_kvcache`` docstring: the cache is
   (batch, seqlen_cache, nheads_k, headdim) and ``cache_seqlens`` gives the
   number of valid keys per batch row.
@@ -32,6 +37,9 @@ Readings where the pages are silent:
 * The backward is the textbook softmax Jacobian: dV = P^T dO, dP = dO V^T,
   Delta_i = sum_j P_ij dP_ij, dS = P * (dP - Delta), dQ = scale dS K,
   dK = scale dS^T Q.  Rows that are fully masked contribute nothing.
+* A causal mask and a window given together keep the keys that both keep
+  (the causal rule caps the right side of the window at 0).  Any negative
+  window side is unbounded, like -1.
 * Varlen packing: tokens of sequence s occupy rows cu[s] .. cu[s+1]-1 of a
   (total, heads, headdim) array; each sequence is an independent problem.
 """
@@ -52,18 +60,28 @@ def kv_head_of(h: int, n_heads_q: int, n_heads_kv: int) -> int:
     return h // group
 
 
-def allowed_mask(len_q: int, len_k: int, causal: bool) -> np.ndarray:
+def allowed_mask(len_q: int, len_k: int, causal: bool, window=(-1, -1)) -> np.ndarray:
     """Boolean (len_q, len_k) matrix, True where query i may attend to key j.
 
     README, ``flash_attn_with_kvcache`` docstring / changelog 2.1: the causal
     mask is aligned to the bottom-right corner, so key j is kept iff
     j <= i + len_k - len_q.  Without ``causal`` every key is kept.
+    README, ``flash_attn_func`` docstring: a sliding window (left, right) keeps
+    only keys in [i + len_k - len_q - left, i + len_k - len_q + right]; a
+    negative side is unbounded.  Both rules together keep the intersection.
     """
     i = np.arange(len_q)[:, None]
     j = np.arange(len_k)[None, :]
-    if not causal:
-        return np.ones((len_q, len_k), dtype=bool)
-    return j <= i + (len_k - len_q)
+    off = len_k - len_q
+    keep = np.ones((len_q, len_k), dtype=bool)
+    if causal:
+        keep &= j <= i + off
+    left, right = window
+    if left >= 0:
+        keep &= j >= i + off - left
+    if right >= 0:
+        keep &= j <= i + off + right
+    return keep
 
 
 def _scores(q: np.ndarray, k: np.ndarray, scale: float, mask: np.ndarray) -> np.ndarray:
@@ -119,7 +137,7 @@ def _check_heads(hq: int, hkv: int) -> int:
     return hq // hkv
 
 
-def mha_forward(q, k, v, scale, causal):
+def mha_forward(q, k, v, scale, causal, window=(-1, -1)):
     """Dense batched attention.
 
     q (B, Sq, Hq, D), k/v (B, Sk, Hkv, D) -> O (B, Sq, Hq, D), LSE (B, Hq, Sq).
@@ -127,7 +145,7 @@ def mha_forward(q, k, v, scale, causal):
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
     _check_heads(Hq, Hkv)
-    mask = allowed_mask(Sq, Sk, causal)
+    mask = allowed_mask(Sq, Sk, causal, window)
     o = np.zeros(q.shape[:3] + (v.shape[3],), dtype=np.float64)
     lse = np.zeros((B, Hq, Sq), dtype=np.float64)
     for b in range(B):
@@ -137,7 +155,7 @@ def mha_forward(q, k, v, scale, causal):
     return o, lse
 
 
-def mha_backward(q, k, v, do, scale, causal):
+def mha_backward(q, k, v, do, scale, causal, window=(-1, -1)):
     """Dense batched backward: returns dQ (like q), dK, dV (like k, v).
 
     With GQA the gradients of a KV head are the sums over the query heads
@@ -146,7 +164,7 @@ def mha_backward(q, k, v, do, scale, causal):
     B, Sq, Hq, D = q.shape
     _, Sk, Hkv, _ = k.shape
     _check_heads(Hq, Hkv)
-    mask = allowed_mask(Sq, Sk, causal)
+    mask = allowed_mask(Sq, Sk, causal, window)
     dq = np.zeros(q.shape, dtype=np.float64)
     dk = np.zeros(k.shape, dtype=np.float64)
     dv = np.zeros(v.shape, dtype=np.float64)
@@ -165,7 +183,7 @@ def _spans(cu):
     return [(int(cu[s]), int(cu[s + 1])) for s in range(len(cu) - 1)]
 
 
-def varlen_forward(q, k, v, cu_q, cu_k, scale, causal):
+def varlen_forward(q, k, v, cu_q, cu_k, scale, causal, window=(-1, -1)):
     """Packed variable-length batch.
 
     q (total_q, Hq, D), k/v (total_k, Hkv, D); sequence s spans rows
@@ -178,7 +196,7 @@ def varlen_forward(q, k, v, cu_q, cu_k, scale, causal):
     o = np.zeros((total_q, Hq, v.shape[2]), dtype=np.float64)
     lse = np.zeros((Hq, total_q), dtype=np.float64)
     for (q0, q1), (k0, k1) in zip(_spans(cu_q), _spans(cu_k)):
-        mask = allowed_mask(q1 - q0, k1 - k0, causal)
+        mask = allowed_mask(q1 - q0, k1 - k0, causal, window)
         for h in range(Hq):
             hk = kv_head_of(h, Hq, Hkv)
             oo, ll, _ = head_forward(q[q0:q1, h, :], k[k0:k1, hk, :], v[k0:k1, hk, :], scale, mask)
@@ -187,7 +205,7 @@ def varlen_forward(q, k, v, cu_q, cu_k, scale, causal):
     return o, lse
 
 
-def varlen_backward(q, k, v, do, cu_q, cu_k, scale, causal):
+def varlen_backward(q, k, v, do, cu_q, cu_k, scale, causal, window=(-1, -1)):
     """Backward of :func:`varlen_forward`; returns dQ, dK, dV in the packed layouts."""
     total_q, Hq, D = q.shape
     Hkv = k.shape[1]
@@ -196,7 +214,7 @@ def varlen_backward(q, k, v, do, cu_q, cu_k, scale, causal):
     dk = np.zeros(k.shape, dtype=np.float64)
     dv = np.zeros(v.shape, dtype=np.float64)
     for (q0, q1), (k0, k1) in zip(_spans(cu_q), _spans(cu_k)):
-        mask = allowed_mask(q1 - q0, k1 - k0, causal)
+        mask = allowed_mask(q1 - q0, k1 - k0, causal, window)
         for h in range(Hq):
             hk = kv_head_of(h, Hq, Hkv)
             gq, gk, gv = head_backward(q[q0:q1, h, :], k[k0:k1, hk, :], v[k0:k1, hk, :], do[q0:q1, h, :], scale, mask)
@@ -206,7 +224,7 @@ def varlen_backward(q, k, v, do, cu_q, cu_k, scale, causal):
     return dq, dk, dv
 
 
-def kvcache_forward(q, k_cache, v_cache, cache_seqlens, scale, causal, rows=None):
+def kvcache_forward(q, k_cache, v_cache, cache_seqlens, scale, causal, rows=None, window=(-1, -1)):
     """Attention of new queries against a contiguous KV cache.
 
     README, ``flash_attn_with_kvcache`` docstring: q (B, Sq, Hq, D); caches
@@ -227,7 +245,7 @@ def kvcache_forward(q, k_cache, v_cache, cache_seqlens, scale, causal, rows=None
         hk = kv_head_of(h, Hq, Hkv)
         kk = np.asarray(k_cache[b, :L, hk, :], dtype=np.float64)
         vv = np.asarray(v_cache[b, :L, hk, :], dtype=np.float64)
-        mask = allowed_mask(Sq, L, causal)
+        mask = allowed_mask(Sq, L, causal, window)
         oo, ll, _ = head_forward(q[b, :, h, :], kk, vv, scale, mask)
         o[b, :, h, :] = oo
         lse[b, h, :] = ll

@@ -302,3 +302,105 @@ def test_merge_of_key_blocks_equals_full_attention():
     om, lm = oracle.merge_lse_partials(parts_l, parts_o)
     np.testing.assert_allclose(om, o, atol=1e-13)
     np.testing.assert_allclose(lm, lse, atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- sliding window
+
+
+@pytest.mark.parametrize("name,Lq,Lk,window", [
+    ("window_mask_q4_k6_l1_r0.txt", 4, 6, (1, 0)),
+    ("window_mask_q5_k3_l0_r1.txt", 5, 3, (0, 1)),
+    ("window_mask_q5_k5_l2_unbounded.txt", 5, 5, (2, -1)),
+])
+def test_window_mask_matches_hand_derived_interval(name, Lq, Lk, window):
+    want = np.array(read_golden(name), dtype=bool)
+    assert np.array_equal(oracle.allowed_mask(Lq, Lk, False, window), want)
+
+
+def test_window_reduces_to_causal_and_full_masks():
+    for Lq, Lk in ((2, 5), (5, 2), (7, 7)):
+        # right side 0 with an unbounded left side is the bottom-right causal mask the pages print
+        assert np.array_equal(oracle.allowed_mask(Lq, Lk, False, (-1, 0)), oracle.allowed_mask(Lq, Lk, True))
+        assert oracle.allowed_mask(Lq, Lk, False, (-1, -1)).all()
+        assert oracle.allowed_mask(Lq, Lk, False, (Lq + Lk, Lq + Lk)).all()
+    want = np.array(read_golden("causal_mask_q2_k5.txt"), dtype=bool)
+    assert np.array_equal(oracle.allowed_mask(2, 5, False, (-1, 0)), want)
+
+
+def test_causal_with_window_keeps_the_intersection():
+    # the reading taken where the pages are silent: both rules apply
+    for Lq, Lk, w in ((6, 9, (2, 3)), (9, 6, (1, 0)), (8, 8, (3, -1))):
+        both = oracle.allowed_mask(Lq, Lk, True, w)
+        assert np.array_equal(both, oracle.allowed_mask(Lq, Lk, True) & oracle.allowed_mask(Lq, Lk, False, w))
+
+
+def _row_interval(i, Lq, Lk, window):
+    # the docstring's interval for query i, clipped to the keys that exist
+    off = Lk - Lq
+    lo = 0 if window[0] < 0 else max(0, i + off - window[0])
+    hi = Lk - 1 if window[1] < 0 else min(Lk - 1, i + off + window[1])
+    return lo, hi
+
+
+def _sliced_rows(q, k, v, scale, window):
+    """Each query row attends, with no mask at all, to the slice of keys its window names
+    (torch fp64 SDPA per row); rows whose slice is empty give 0 / -inf."""
+    Lq, Lk = q.shape[0], k.shape[0]
+    outs, lses = [], []
+    for i in range(Lq):
+        lo, hi = _row_interval(i, Lq, Lk, window)
+        if hi < lo:
+            outs.append(torch.zeros(v.shape[1], dtype=torch.float64))
+            lses.append(torch.tensor(-math.inf, dtype=torch.float64))
+            continue
+        ks, vs = k[lo:hi + 1], v[lo:hi + 1]
+        o = torch.nn.functional.scaled_dot_product_attention(q[i:i + 1][None], ks[None], vs[None], scale=scale)
+        outs.append(o[0, 0])
+        lses.append(torch.logsumexp(scale * (ks @ q[i]), dim=0))
+    return torch.stack(outs), torch.stack(lses)
+
+
+@pytest.mark.parametrize("Lq,Lk,window", [(13, 13, (3, 0)), (9, 14, (2, 1)), (14, 9, (0, 2)),
+                                          (11, 11, (-1, 2)), (10, 10, (4, -1)), (6, 6, (0, 0))])
+def test_window_forward_matches_sliced_sdpa(Lq, Lk, window):
+    q, k, v = rnd(Lq, 8), rnd(Lk, 8), rnd(Lk, 8)
+    o, lse, _ = oracle.head_forward(q, k, v, 0.4, oracle.allowed_mask(Lq, Lk, False, window))
+    o_ref, lse_ref = _sliced_rows(*(torch.from_numpy(x) for x in (q, k, v)), 0.4, window)
+    np.testing.assert_allclose(o, o_ref.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(np.isneginf(lse), np.isneginf(lse_ref.numpy()))
+    fin = np.isfinite(lse)
+    np.testing.assert_allclose(lse[fin], lse_ref.numpy()[fin], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("Lq,Lk,window", [(12, 12, (3, 0)), (8, 13, (2, 1)), (13, 8, (1, 3))])
+def test_window_backward_matches_sliced_autograd(Lq, Lk, window):
+    B, Hq, Hkv, D = 1, 4, 2, 8
+    q, k, v, do = rnd(B, Lq, Hq, D), rnd(B, Lk, Hkv, D), rnd(B, Lk, Hkv, D), rnd(B, Lq, Hq, D)
+    dq, dk, dv = oracle.mha_backward(q, k, v, do, 0.35, False, window)
+    tq, tk, tv = (torch.from_numpy(x.copy()).requires_grad_() for x in (q, k, v))
+    loss = 0
+    for h in range(Hq):
+        hk = h // (Hq // Hkv)
+        o, _ = _sliced_rows(tq[0, :, h], tk[0, :, hk], tv[0, :, hk], 0.35, window)
+        loss = loss + (o * torch.from_numpy(do[0, :, h])).sum()
+    loss.backward()
+    for got, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-11)
+
+
+def test_window_varlen_equals_per_sequence_dense():
+    lens = [5, 17, 1, 9]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    q, k, v, do = rnd(T, 2, 8), rnd(T, 1, 8), rnd(T, 1, 8), rnd(T, 2, 8)
+    w = (3, 1)
+    o, lse = oracle.varlen_forward(q, k, v, cu, cu, 0.3, True, w)
+    dq, dk, dv = oracle.varlen_backward(q, k, v, do, cu, cu, 0.3, True, w)
+    for a, b in zip(cu[:-1], cu[1:]):
+        od, ld = oracle.mha_forward(q[None, a:b], k[None, a:b], v[None, a:b], 0.3, True, w)
+        gq, gk, gv = oracle.mha_backward(q[None, a:b], k[None, a:b], v[None, a:b], do[None, a:b], 0.3, True, w)
+        np.testing.assert_array_equal(o[a:b], od[0])
+        np.testing.assert_array_equal(lse[:, a:b], ld[0])
+        np.testing.assert_array_equal(dq[a:b], gq[0])
+        np.testing.assert_array_equal(dk[a:b], gk[0])
+        np.testing.assert_array_equal(dv[a:b], gv[0])

@@ -13,10 +13,29 @@ import oracle.attention as A
 from tests import test_oracle as pins
 
 
-def _mask_top_left(len_q, len_k, causal):
+def _mask_top_left(len_q, len_k, causal, window=(-1, -1)):
     i = np.arange(len_q)[:, None]
     j = np.arange(len_k)[None, :]
     return np.ones((len_q, len_k), bool) if not causal else (j <= i)
+
+
+def _window_left_off_by_one(len_q, len_k, causal, window=(-1, -1)):
+    # the left edge of the window taken one key too far
+    left, right = window
+    return _ORIG_MASK(len_q, len_k, causal, (left + 1 if left >= 0 else left, right))
+
+
+def _window_top_left(len_q, len_k, causal, window=(-1, -1)):
+    # the window anchored at the diagonal i = j instead of the bottom-right corner
+    m = _ORIG_MASK(len_q, len_k, causal)
+    i = np.arange(len_q)[:, None]
+    j = np.arange(len_k)[None, :]
+    left, right = window
+    if left >= 0:
+        m &= j >= i - left
+    if right >= 0:
+        m &= j <= i + right
+    return m
 
 
 def _gqa_modulo(h, hq, hkv):
@@ -65,6 +84,7 @@ def _bwd_dv_from_do_transposed(q, k, v, do, scale, mask):
 
 
 _ORIG_FWD = A.head_forward
+_ORIG_MASK = A.allowed_mask
 _ORIG_BWD = A.head_backward
 
 
@@ -100,3 +120,18 @@ def test_lse_missing_max_is_caught(monkeypatch):
 def test_backward_mutants_are_caught(monkeypatch, mutant):
     monkeypatch.setattr(A, "head_backward", mutant)
     _fails(pins.test_backward_matches_torch_autograd, False, 9, 9, 2, 2)
+
+
+@pytest.mark.parametrize("mutant", [_window_left_off_by_one, _window_top_left])
+def test_window_mask_mutants_are_caught(monkeypatch, mutant):
+    monkeypatch.setattr(A, "allowed_mask", mutant)
+    monkeypatch.setattr(oracle, "allowed_mask", mutant)
+    caught = 0
+    for args in (("window_mask_q4_k6_l1_r0.txt", 4, 6, (1, 0)), ("window_mask_q5_k3_l0_r1.txt", 5, 3, (0, 1)),
+                 ("window_mask_q5_k5_l2_unbounded.txt", 5, 5, (2, -1))):
+        try:
+            pins.test_window_mask_matches_hand_derived_interval(*args)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+    _fails(pins.test_window_forward_matches_sliced_sdpa, 9, 14, (2, 1))
