@@ -31,6 +31,7 @@ EXPORTS = (
     "fa_set_wait_timeout_ns", "fa_debug_wait_timeout_selftest", "fa_debug_umma_selftest",
     "fa_profile_begin", "fa_profile_read",
     "fa_fwd_kvcache_noalloc", "fa_fwd_kvcache_noalloc_scratch_bytes", "fa_debug_exp2_selftest",
+    "fa_fwd_ex", "fa_bwd_ex", "fa_varlen_fwd_ex", "fa_varlen_bwd_ex",
 )
 
 FA_KERNEL_FWD = 0
@@ -64,6 +65,10 @@ _SIGS = {
     "fa_fwd_kvcache_noalloc": (_I, [_P] * 6 + [_I] * 6 + [_F, _I, _I, _P]),
     "fa_fwd_kvcache_noalloc_scratch_bytes": (_Z, []),
     "fa_debug_exp2_selftest": (_I, [_P, _P, _I, _P]),
+    "fa_fwd_ex": (_I, [_P] * 5 + [_I] * 6 + [_F, _I, _I, _I, _P, _Z, _P]),
+    "fa_bwd_ex": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _I, _I, _P, _Z, _P]),
+    "fa_varlen_fwd_ex": (_I, [_P] * 7 + [_I] * 8 + [_F, _I, _I, _I, _P, _Z, _P]),
+    "fa_varlen_bwd_ex": (_I, [_P] * 11 + [_I] * 8 + [_F, _I, _I, _I, _I, _P, _Z, _P]),
 }
 
 _lib = None
@@ -166,6 +171,40 @@ def fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, out, lse, B, Hq, Hkv, Sq,
     return load().fa_fwd_kvcache(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens), _ptr(out), _ptr(lse),
                                  B, Hq, Hkv, Sq, cache_capacity, D, float(softmax_scale), int(bool(causal)),
                                  int(num_splits), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def fa_fwd_ex(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, window_left, window_right,
+              workspace=None, workspace_bytes=0, stream=None) -> int:
+    return load().fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Sq, Sk, D,
+                            float(softmax_scale), int(bool(causal)), int(window_left), int(window_right),
+                            _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def fa_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, window_left,
+              window_right, deterministic, workspace, workspace_bytes, stream=None) -> int:
+    return load().fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                            _ptr(dv), B, Hq, Hkv, Sq, Sk, D, float(softmax_scale), int(bool(causal)),
+                            int(window_left), int(window_right), int(bool(deterministic)), _ptr(workspace),
+                            workspace_bytes, _stream(stream))
+
+
+def fa_varlen_fwd_ex(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
+                     total_k, Hq, Hkv, D, softmax_scale, causal, window_left, window_right, workspace=None,
+                     workspace_bytes=0, stream=None) -> int:
+    return load().fa_varlen_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens_q),
+                                   _ptr(cu_seqlens_k), num_seqs, max_seqlen_q, max_seqlen_k, total_q, total_k, Hq,
+                                   Hkv, D, float(softmax_scale), int(bool(causal)), int(window_left),
+                                   int(window_right), _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def fa_varlen_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q,
+                     max_seqlen_k, total_q, total_k, Hq, Hkv, D, softmax_scale, causal, window_left, window_right,
+                     deterministic, workspace, workspace_bytes, stream=None) -> int:
+    return load().fa_varlen_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                                   _ptr(dv), _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), num_seqs, max_seqlen_q,
+                                   max_seqlen_k, total_q, total_k, Hq, Hkv, D, float(softmax_scale),
+                                   int(bool(causal)), int(window_left), int(window_right), int(bool(deterministic)),
+                                   _ptr(workspace), workspace_bytes, _stream(stream))
 
 
 def fa_get_device_status(stream=None) -> int:

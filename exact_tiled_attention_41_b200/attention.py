@@ -7,6 +7,9 @@ Shapes follow the flash-attention README (flash_attn_func, flash_attn_varlen_fun
 flash_attn_with_kvcache docstrings): q (B, Sq, Hq, D), k/v (B, Sk, Hkv, D); varlen
 q (total_q, Hq, D) with int32 cu_seqlens; caches (B, capacity, Hkv, D).
 softmax_scale defaults to 1/sqrt(D) (README, "How to use FlashAttention").
+window_size = (left, right) is the sliding window of the flash_attn_func docstring
+(-1 = unbounded side); deterministic selects the backward whose dq does not depend
+on the order of float additions.
 """
 
 from __future__ import annotations
@@ -41,7 +44,12 @@ def _workspace(nbytes: int, device) -> torch.Tensor | None:
     return torch.empty(nbytes, dtype=torch.uint8, device=device)
 
 
-def flash_attn_func(q, k, v, softmax_scale=None, causal=False):
+def _window(window_size):
+    left, right = window_size
+    return int(left), int(right)
+
+
+def flash_attn_func(q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1)):
     """Forward: returns (out (B, Sq, Hq, D) bf16, lse (B, Hq, Sq) fp32)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
@@ -50,11 +58,12 @@ def flash_attn_func(q, k, v, softmax_scale=None, causal=False):
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
     out = torch.empty_like(q)
     lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    _raise(abi.fa_fwd(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal), "fa_fwd")
+    _raise(abi.fa_fwd_ex(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, *_window(window_size)), "fa_fwd")
     return out, lse
 
 
-def flash_attn_backward(dout, q, k, v, out, lse, softmax_scale=None, causal=False):
+def flash_attn_backward(dout, q, k, v, out, lse, softmax_scale=None, causal=False, window_size=(-1, -1),
+                        deterministic=False):
     """Backward: returns (dq, dk, dv) shaped like q, k, v."""
     for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")):
         _check(t, n)
@@ -65,12 +74,13 @@ def flash_attn_backward(dout, q, k, v, out, lse, softmax_scale=None, causal=Fals
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     nb = abi.fa_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D)
     ws = _workspace(nb, q.device)
-    _raise(abi.fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, scale, causal, ws, nb), "fa_bwd")
+    _raise(abi.fa_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, scale, causal,
+                         *_window(window_size), deterministic, ws, nb), "fa_bwd")
     return dq, dk, dv
 
 
 def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, softmax_scale=None,
-                           causal=False):
+                           causal=False, window_size=(-1, -1)):
     """Packed forward: returns (out (total_q, Hq, D), lse (Hq, total_q))."""
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check(t, n)
@@ -82,13 +92,13 @@ def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, ma
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
     out = torch.empty_like(q)
     lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
-    _raise(abi.fa_varlen_fwd(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q, max_seqlen_k,
-                             total_q, total_k, Hq, Hkv, D, scale, causal), "fa_varlen_fwd")
+    _raise(abi.fa_varlen_fwd_ex(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q, max_seqlen_k,
+                                total_q, total_k, Hq, Hkv, D, scale, causal, *_window(window_size)), "fa_varlen_fwd")
     return out, lse
 
 
 def flash_attn_varlen_backward(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k,
-                               softmax_scale=None, causal=False):
+                               softmax_scale=None, causal=False, window_size=(-1, -1), deterministic=False):
     for t, n in ((dout, "dout"), (q, "q"), (k, "k"), (v, "v"), (out, "out")):
         _check(t, n)
     _check(lse, "lse", torch.float32)
@@ -99,8 +109,9 @@ def flash_attn_varlen_backward(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     nb = abi.fa_varlen_bwd_workspace_size(nseq, total_q, total_k, Hq, Hkv, D)
     ws = _workspace(nb, q.device)
-    _raise(abi.fa_varlen_bwd(q, k, v, out, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q,
-                             max_seqlen_k, total_q, total_k, Hq, Hkv, D, scale, causal, ws, nb), "fa_varlen_bwd")
+    _raise(abi.fa_varlen_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q,
+                                max_seqlen_k, total_q, total_k, Hq, Hkv, D, scale, causal, *_window(window_size),
+                                deterministic, ws, nb), "fa_varlen_bwd")
     return dq, dk, dv
 
 
@@ -123,17 +134,19 @@ def flash_attn_with_kvcache(q, k_cache, v_cache, cache_seqlens, softmax_scale=No
 
 
 class FlashAttnFunction(torch.autograd.Function):
-    """Autograd wrapper: forward = fa_fwd, backward = fa_bwd."""
+    """Autograd wrapper: forward = fa_fwd_ex, backward = fa_bwd_ex."""
 
     @staticmethod
-    def forward(ctx, q, k, v, softmax_scale=None, causal=False):
-        out, lse = flash_attn_func(q, k, v, softmax_scale, causal)
+    def forward(ctx, q, k, v, softmax_scale=None, causal=False, window_size=(-1, -1), deterministic=False):
+        out, lse = flash_attn_func(q, k, v, softmax_scale, causal, window_size)
         ctx.save_for_backward(q, k, v, out, lse)
         ctx.softmax_scale, ctx.causal = softmax_scale, causal
+        ctx.window_size, ctx.deterministic = window_size, deterministic
         return out
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, out, lse = ctx.saved_tensors
-        dq, dk, dv = flash_attn_backward(dout.contiguous(), q, k, v, out, lse, ctx.softmax_scale, ctx.causal)
-        return dq, dk, dv, None, None
+        dq, dk, dv = flash_attn_backward(dout.contiguous(), q, k, v, out, lse, ctx.softmax_scale, ctx.causal,
+                                         ctx.window_size, ctx.deterministic)
+        return dq, dk, dv, None, None, None, None

@@ -93,6 +93,18 @@ static int check_heads(int Hq, int Hkv, int D, float scale) {
     return FA_OK;
 }
 
+// Sequence lengths are bounded by 2^30 so that row +- window arithmetic stays inside int32 in the kernels.
+static const int kMaxSeqlen = 1 << 30;
+
+// Window sides as the kernels take them: -1 = unbounded; a causal mask caps the right side at 0
+// (the keys kept are those both rules keep).  Any negative side counts as unbounded, and so does a
+// side of 2^30 or more: with j - (i + Sk - Sq) in [1 - Sk, Sq - 1] it never excludes a key.
+static void window_sides(int causal, int window_left, int window_right, int* wl, int* wr) {
+    *wl = (window_left < 0 || window_left >= kMaxSeqlen) ? -1 : window_left;
+    *wr = (window_right < 0 || window_right >= kMaxSeqlen) ? -1 : window_right;
+    if (causal) *wr = 0;
+}
+
 static int check_tokens(long long tokens, int H, int D) {
     // element indices are formed in 64-bit, token coordinates of tile loads in int32
     if (tokens > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
@@ -139,6 +151,7 @@ static int validate_dense(const void* q, const void* k, const void* v, int B, in
                           float scale) {
     if (q == nullptr || k == nullptr || v == nullptr) return FA_ERR_INVALID_ARG;
     if (B <= 0 || Sq <= 0 || Sk <= 0) return FA_ERR_INVALID_ARG;
+    if (Sq > kMaxSeqlen || Sk > kMaxSeqlen) return FA_ERR_UNSUPPORTED;
     int st = check_heads(Hq, Hkv, D, scale);
     if (st != FA_OK) return st;
     if ((st = check_tokens(static_cast<long long>(B) * Sq, Hq, D)) != FA_OK) return st;
@@ -148,7 +161,7 @@ static int validate_dense(const void* q, const void* k, const void* v, int B, in
 }
 
 static Problem dense_problem(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int Sq, int Sk,
-                             int D, float scale, int causal) {
+                             int D, float scale, int causal, int window_left, int window_right) {
     Problem pr;
     pr.q = q;
     pr.k = k;
@@ -164,7 +177,7 @@ static Problem dense_problem(const void* q, const void* k, const void* v, int B,
     pr.Hkv = Hkv;
     pr.D = D;
     pr.scale = scale;
-    pr.causal = causal ? 1 : 0;
+    window_sides(causal, window_left, window_right, &pr.wl, &pr.wr);
     pr.lse_sB = static_cast<long long>(Hq) * Sq;
     pr.lse_sH = Sq;
     pr.lse_sT = 0;
@@ -173,6 +186,13 @@ static Problem dense_problem(const void* q, const void* k, const void* v, int B,
 
 int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq, int Sk,
            int D, float softmax_scale, int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    return fa_fwd_ex(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, -1, -1, workspace,
+                     workspace_bytes, stream);
+}
+
+int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
+              int Sk, int D, float softmax_scale, int causal, int window_left, int window_right, void* workspace,
+              size_t workspace_bytes, fa_stream_t stream) {
     (void)workspace;
     (void)workspace_bytes;
     int st = validate_dense(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale);
@@ -181,7 +201,7 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
     if (!aligned16(out) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
     Device dev;
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
-    Problem pr = dense_problem(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal);
+    Problem pr = dense_problem(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, window_left, window_right);
     return launch_fwd(pr, out, lse, dev, static_cast<cudaStream_t>(stream));
 }
 
@@ -196,6 +216,14 @@ size_t fa_bwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D) {
 int fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse, void* dq,
            void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int D, float softmax_scale, int causal,
            void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    return fa_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, -1, -1, 0,
+                     workspace, workspace_bytes, stream);
+}
+
+int fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+              void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq, int Sk, int D, float softmax_scale,
+              int causal, int window_left, int window_right, int deterministic, void* workspace,
+              size_t workspace_bytes, fa_stream_t stream) {
     int st = validate_dense(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale);
     if (st != FA_OK) return st;
     if (!out || !dout || !lse || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
@@ -205,8 +233,9 @@ int fa_bwd(const void* q, const void* k, const void* v, const void* out, const v
     if (workspace_bytes < fa_bwd_workspace_size(B, Hq, Hkv, Sq, Sk, D)) return FA_ERR_WORKSPACE;
     Device dev;
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
-    Problem pr = dense_problem(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal);
-    return launch_bwd(pr, out, dout, lse, dq, dk, dv, workspace, dev, static_cast<cudaStream_t>(stream));
+    Problem pr = dense_problem(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, window_left, window_right);
+    return launch_bwd(pr, out, dout, lse, dq, dk, dv, workspace, deterministic != 0, dev,
+                      static_cast<cudaStream_t>(stream));
 }
 
 // ----------------------------------------------------------------------- varlen
@@ -215,6 +244,7 @@ static int validate_varlen(const void* q, const void* k, const void* v, const in
                            float scale) {
     if (!q || !k || !v || !cu_q || !cu_k) return FA_ERR_INVALID_ARG;
     if (num_seqs <= 0 || max_q <= 0 || max_k <= 0 || total_q <= 0 || total_k <= 0) return FA_ERR_INVALID_ARG;
+    if (max_q > kMaxSeqlen || max_k > kMaxSeqlen) return FA_ERR_UNSUPPORTED;
     int st = check_heads(Hq, Hkv, D, scale);
     if (st != FA_OK) return st;
     if ((st = check_tokens(total_q, Hq, D)) != FA_OK) return st;
@@ -226,7 +256,7 @@ static int validate_varlen(const void* q, const void* k, const void* v, const in
 
 static Problem varlen_problem(const void* q, const void* k, const void* v, const int32_t* cu_q, const int32_t* cu_k,
                               int num_seqs, int max_q, int max_k, int total_q, int total_k, int Hq, int Hkv, int D,
-                              float scale, int causal) {
+                              float scale, int causal, int window_left, int window_right) {
     Problem pr;
     pr.q = q;
     pr.k = k;
@@ -242,7 +272,7 @@ static Problem varlen_problem(const void* q, const void* k, const void* v, const
     pr.Hkv = Hkv;
     pr.D = D;
     pr.scale = scale;
-    pr.causal = causal ? 1 : 0;
+    window_sides(causal, window_left, window_right, &pr.wl, &pr.wr);
     pr.lse_sB = 0;
     pr.lse_sH = total_q;
     pr.lse_sT = 1;
@@ -255,6 +285,15 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* out, float*
                   const int32_t* cu_seqlens_k, int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q,
                   int total_k, int Hq, int Hkv, int D, float softmax_scale, int causal, void* workspace,
                   size_t workspace_bytes, fa_stream_t stream) {
+    return fa_varlen_fwd_ex(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k,
+                            total_q, total_k, Hq, Hkv, D, softmax_scale, causal, -1, -1, workspace, workspace_bytes,
+                            stream);
+}
+
+int fa_varlen_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, const int32_t* cu_seqlens_q,
+                     const int32_t* cu_seqlens_k, int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q,
+                     int total_k, int Hq, int Hkv, int D, float softmax_scale, int causal, int window_left,
+                     int window_right, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
     (void)workspace;
     (void)workspace_bytes;
     int st = validate_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q, total_k,
@@ -265,7 +304,7 @@ int fa_varlen_fwd(const void* q, const void* k, const void* v, void* out, float*
     Device dev;
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
     Problem pr = varlen_problem(q, k, v, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
-                                total_k, Hq, Hkv, D, softmax_scale, causal);
+                                total_k, Hq, Hkv, D, softmax_scale, causal, window_left, window_right);
     return launch_fwd(pr, out, lse, dev, static_cast<cudaStream_t>(stream));
 }
 
@@ -281,6 +320,16 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* out, 
                   void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int num_seqs,
                   int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv, int D,
                   float softmax_scale, int causal, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    return fa_varlen_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q,
+                            max_seqlen_k, total_q, total_k, Hq, Hkv, D, softmax_scale, causal, -1, -1, 0, workspace,
+                            workspace_bytes, stream);
+}
+
+int fa_varlen_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout, const float* lse,
+                     void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                     int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int Hq, int Hkv,
+                     int D, float softmax_scale, int causal, int window_left, int window_right, int deterministic,
+                     void* workspace, size_t workspace_bytes, fa_stream_t stream) {
     int st = validate_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q, total_k,
                              Hq, Hkv, D, softmax_scale);
     if (st != FA_OK) return st;
@@ -292,8 +341,9 @@ int fa_varlen_bwd(const void* q, const void* k, const void* v, const void* out, 
     Device dev;
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
     Problem pr = varlen_problem(q, k, v, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
-                                total_k, Hq, Hkv, D, softmax_scale, causal);
-    return launch_bwd(pr, out, dout, lse, dq, dk, dv, workspace, dev, static_cast<cudaStream_t>(stream));
+                                total_k, Hq, Hkv, D, softmax_scale, causal, window_left, window_right);
+    return launch_bwd(pr, out, dout, lse, dq, dk, dv, workspace, deterministic != 0, dev,
+                      static_cast<cudaStream_t>(stream));
 }
 
 // ----------------------------------------------------------------------- KV-cache decode

@@ -14,8 +14,8 @@
 //   2. main kernel, one persistent CTA per SM, KV-tile stationary: a work unit
 //      is (sequence, KV head, 128-key tile); it loops over the 128-row query
 //      tiles of every query head that reads the KV head (so dK and dV of GQA
-//      need no atomics) and, for causal masks, only over query tiles that can
-//      see the key tile.  Roles (16 warps, registers redistributed with setmaxnreg):
+//      need no atomics) and only over the query tiles that can see the key
+//      tile (causal masks and sliding windows cut the range at both ends).  Roles (16 warps, registers redistributed with setmaxnreg):
 //        warps 0-7   two compute warpgroups, thread = key row, each owning 64 of
 //                    the 128 query columns: P^T, dS^T from S^T and dP^T in tensor
 //                    memory (written back as bf16, dS^T also to shared memory);
@@ -51,7 +51,7 @@ struct BwdParams {
     int num_seqs, Sq, Sk, Tq, Tk, Hq, Hkv, group;
     int n_blocks, num_units;
     float scale, scale_log2;
-    int causal;
+    int wl, wr;             // window sides, -1 = unbounded; a causal mask is wr = 0
     unsigned long long timeout_ns;
     int* status;
 };
@@ -75,8 +75,8 @@ __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
         t.Lk = __ldg(p.cu_k + t.b + 1) - t.k_start;
         t.q_start = max(t.q_start, 0);
         t.k_start = max(t.k_start, 0);
-        t.Lq = max(min(t.Lq, p.Tq - t.q_start), 0);
-        t.Lk = max(min(t.Lk, p.Tk - t.k_start), 0);
+        t.Lq = max(min(min(t.Lq, p.Tq - t.q_start), 1 << 30), 0);   // at most 2^30 tokens per sequence
+        t.Lk = max(min(min(t.Lk, p.Tk - t.k_start), 1 << 30), 0);
     } else {
         t.q_start = t.b * p.Sq;
         t.Lq = p.Sq;
@@ -85,14 +85,20 @@ __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
     }
     t.n0 = n * 128;
     t.skip = t.n0 >= t.Lk;
-    int m_start = 0;
-    if (p.causal) {
-        const int first_row = t.n0 - (t.Lk - t.Lq);   // first query row that sees key n0
-        m_start = first_row > 0 ? first_row / 128 : 0;
+    // query rows that see some key of n0 .. n0+127: key j is allowed for row i iff
+    // i + off - wl <= j <= i + off + wr, i.e. j - off - wr <= i <= j - off + wl
+    // (lengths <= 2^30 and window sides < 2^30 keep every term inside int32)
+    const int off = t.Lk - t.Lq;
+    int r_lo = 0, r_hi = t.Lq - 1;
+    if (p.wr >= 0) r_lo = max(r_lo, t.n0 - off - p.wr);
+    if (p.wl >= 0) r_hi = min(r_hi, min(t.n0 + 127, t.Lk - 1) - off + p.wl);
+    if (t.skip || r_hi < r_lo) {
+        t.m_start = 0;
+        t.n_m = 0;
+    } else {
+        t.m_start = r_lo / 128;
+        t.n_m = r_hi / 128 + 1 - t.m_start;
     }
-    const int m_end = (t.Lq + 127) / 128;
-    t.m_start = m_start;
-    t.n_m = m_end > m_start ? m_end - m_start : 0;
     t.n_it = t.n_m * p.group;
     return t;
 }
@@ -370,7 +376,12 @@ __global__ void __launch_bounds__(512, 1)
                 }
                 continue;
             }
-            const int off = t.Lk - t.Lq;
+            // this key row is seen by query rows q_lo .. q_hi of the sequence
+            // (a key row past the sequence is seen by none: an empty range)
+            int q_lo = -0x40000000, q_hi = 0x40000000;
+            if (p.wr >= 0) q_lo = kj - (t.Lk - t.Lq) - p.wr;
+            if (p.wl >= 0) q_hi = kj - (t.Lk - t.Lq) + p.wl;
+            if (!kvalid) q_lo = 0x40000000;
             for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
                 const int m0 = (t.m_start + it % t.n_m) * 128;
                 const int st = q_it % ST;
@@ -401,9 +412,9 @@ __global__ void __launch_bounds__(512, 1)
                     : "r"(static_cast<uint32_t>(got))
                     : "memory");
                 if (!all_got) { ok = false; break; }
-                // key kj may be seen by query row qi iff kj <= qi + off  <=>  qi >= kj - off
-                const int qmin = p.causal ? kj - off - m0 : -0x40000000;   // first allowed local query column
-                const bool full_row = kvalid && qmin <= 64 * gq;
+                // allowed local query columns of this tile: qmin .. qmax
+                const int qmin = q_lo - m0, qmax = q_hi - m0;
+                const bool full_row = qmin <= 64 * gq && qmax >= 64 * gq + 63;
                 const bool any_mask = __any_sync(0xffffffffu, !full_row);
                 const float* lse_t = sLSE + st * 128 + 64 * gq;
                 const float* del_t = sDel + st * 128 + 64 * gq;
@@ -426,8 +437,8 @@ __global__ void __launch_bounds__(512, 1)
                             float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
                             if (any_mask) {
                                 const int qc = 64 * gq + half * 32 + e + x;
-                                pr.x = (kvalid && qc >= qmin) ? pr.x : 0.f;
-                                pr.y = (kvalid && qc + 1 >= qmin) ? pr.y : 0.f;
+                                pr.x = (qc >= qmin && qc <= qmax) ? pr.x : 0.f;
+                                pr.y = (qc + 1 >= qmin && qc + 1 <= qmax) ? pr.y : 0.f;
                             }
                             const float2 ds = fmul2(pr, fadd2(dv, make_float2(-dla, -dlb)));
                             pp[(e + x) / 2] = pack_bf16x2(pr.x, pr.y);
@@ -631,7 +642,8 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     p.num_units = static_cast<int>(units);
     p.scale = pr.scale;
     p.scale_log2 = pr.scale * 1.4426950408889634f;
-    p.causal = pr.causal;
+    p.wl = pr.wl;
+    p.wr = pr.wr;
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
 
@@ -678,7 +690,8 @@ static int run_bwd256(const Problem& pr, const void* out, const void* dout, cons
 }
 
 int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk, void* dv,
-               void* workspace, const Device& dev, cudaStream_t stream) {
+               void* workspace, bool deterministic, const Device& dev, cudaStream_t stream) {
+    if (deterministic) return 2;
     switch (pr.D) {
         case 64: return run_bwd<64>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
         case 128: return run_bwd<128>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);

@@ -37,7 +37,7 @@ struct B256Params {
     int num_seqs, Sq, Sk, Tq, Tk, Hq, Hkv, group;
     int num_units;
     float scale, scale_log2;
-    int causal;
+    int wl, wr;             // window sides, -1 = unbounded; a causal mask is wr = 0
     unsigned long long timeout_ns;
     int* status;
 };
@@ -59,8 +59,8 @@ __device__ __forceinline__ U256 decode_u256(const B256Params& p, int u) {
     if (p.cu_q != nullptr) {
         t.q_start = max(__ldg(p.cu_q + t.b), 0);
         t.k_start = max(__ldg(p.cu_k + t.b), 0);
-        t.Lq = max(min(__ldg(p.cu_q + t.b + 1) - t.q_start, p.Tq - t.q_start), 0);
-        t.Lk = max(min(__ldg(p.cu_k + t.b + 1) - t.k_start, p.Tk - t.k_start), 0);
+        t.Lq = max(min(min(__ldg(p.cu_q + t.b + 1) - t.q_start, p.Tq - t.q_start), 1 << 30), 0);
+        t.Lk = max(min(min(__ldg(p.cu_k + t.b + 1) - t.k_start, p.Tk - t.k_start), 1 << 30), 0);
     } else {
         t.q_start = t.b * p.Sq;
         t.Lq = p.Sq;
@@ -69,14 +69,19 @@ __device__ __forceinline__ U256 decode_u256(const B256Params& p, int u) {
     }
     t.n0 = n * 128;
     t.skip = t.n0 >= t.Lk;
-    int m_start = 0;
-    if (p.causal) {
-        const int first_row = t.n0 - (t.Lk - t.Lq);
-        m_start = first_row > 0 ? first_row / 64 : 0;
+    // query rows that see some key of the tile (key j allowed for row i iff j - off - wr <= i <= j - off + wl)
+    // (lengths <= 2^30 and window sides < 2^30 keep every term inside int32)
+    const int off = t.Lk - t.Lq;
+    int r_lo = 0, r_hi = t.Lq - 1;
+    if (p.wr >= 0) r_lo = max(r_lo, t.n0 - off - p.wr);
+    if (p.wl >= 0) r_hi = min(r_hi, min(t.n0 + 127, t.Lk - 1) - off + p.wl);
+    if (t.skip || r_hi < r_lo) {
+        t.m_start = 0;
+        t.n_m = 0;
+    } else {
+        t.m_start = r_lo / 64;
+        t.n_m = r_hi / 64 + 1 - t.m_start;
     }
-    const int m_end = (t.Lq + 63) / 64;
-    t.m_start = m_start;
-    t.n_m = m_end > m_start ? m_end - m_start : 0;
     t.n_it = t.n_m * p.group;
     return t;
 }
@@ -318,7 +323,10 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 continue;
             }
-            const int off = t.Lk - t.Lq;
+            // this key row is seen by query rows q_lo .. q_hi of the sequence
+            int q_lo = -0x40000000, q_hi = 0x40000000;
+            if (p.wr >= 0) q_lo = kj - (t.Lk - t.Lq) - p.wr;
+            if (p.wl >= 0) q_hi = kj - (t.Lk - t.Lq) + p.wl;
             for (int it = 0; it < t.n_it; ++it, ++q_it) {
                 const int m0 = (t.m_start + it % t.n_m) * 64;
                 if (!mbar_wait(s_full, q_it & 1, w)) { ok = false; break; }
@@ -333,8 +341,8 @@ __global__ void __launch_bounds__(384, 1)
                 reg_tie(sa[1]);
                 reg_tie(da[0]);
                 reg_tie(da[1]);
-                const int qmin = p.causal ? kj - off - m0 : -0x40000000;
-                const bool any_mask = __any_sync(0xffffffffu, !(kvalid && qmin <= 0));
+                const int qmin = q_lo - m0, qmax = q_hi - m0;
+                const bool any_mask = __any_sync(0xffffffffu, !(kvalid && qmin <= 0 && qmax >= 63));
                 const float2 c2v = make_float2(c2, c2);
                 uint8_t* ds_row = smem + C::OFF_DS + r * 128;
 #pragma unroll
@@ -348,8 +356,8 @@ __global__ void __launch_bounds__(384, 1)
                         const float2 a = ffma2(sv, c2v, make_float2(-sLSE[qc], -sLSE[qc + 1]));
                         float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
                         if (any_mask) {
-                            pr.x = (kvalid && qc >= qmin) ? pr.x : 0.f;
-                            pr.y = (kvalid && qc + 1 >= qmin) ? pr.y : 0.f;
+                            pr.x = (kvalid && qc >= qmin && qc <= qmax) ? pr.x : 0.f;
+                            pr.y = (kvalid && qc + 1 >= qmin && qc + 1 <= qmax) ? pr.y : 0.f;
                         }
                         const float2 ds = fmul2(pr, fadd2(dv, make_float2(-sDel[qc], -sDel[qc + 1])));
                         pp[e / 2] = pack_bf16x2(pr.x, pr.y);
@@ -462,7 +470,8 @@ int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, c
     p.num_units = static_cast<int>(units);
     p.scale = pr.scale;
     p.scale_log2 = pr.scale * 1.4426950408889634f;
-    p.causal = pr.causal;
+    p.wl = pr.wl;
+    p.wr = pr.wr;
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
     static bool set[64] = {};

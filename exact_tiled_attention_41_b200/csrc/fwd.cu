@@ -23,7 +23,10 @@
 //   * work units (sequence, head, block of NQ*128 query rows) are listed
 //     heaviest first (query blocks with most KV tiles first for causal masks)
 //     and dealt to the persistent CTAs in boustrophedon order (snake_unit);
-//     causal blocks stop at the last KV tile they can see.
+//     each query tile only visits the KV tiles its mask can reach: causal
+//     blocks stop at the last KV tile they can see, and a sliding window
+//     (README, flash_attn_func docstring: query i keeps the keys in
+//     [i + Sk - Sq - left, i + Sk - Sq + right]) also starts late.
 //
 // Exactness of the deferred rescale: P, l and O are all taken against the same
 // reference value m_ref of the row, which is only raised when a tile's max
@@ -47,7 +50,7 @@ struct FwdParams {
     int num_seqs, Sq, Sk, Tq, Tk, Hq, Hkv, group;
     int m_blocks, num_units;
     float scale_log2;
-    int causal;
+    int wl, wr;   // window sides, -1 = unbounded; a causal mask is wr = 0
     long long lse_sB, lse_sH;
     int lse_sT;
     unsigned long long timeout_ns;
@@ -55,12 +58,17 @@ struct FwdParams {
 };
 
 struct Unit {
-    int b, h, q_start, k_start, Lq, Lk, q0, n_kv;
-    int n_tile[2];   // KV tiles seen by query tile 0 / 1 (0: the tile has no row inside the sequence)
+    int b, h, q_start, k_start, Lq, Lk, q0;
+    int kv0, n_kv;   // the unit loads KV tiles kv0 .. kv0 + n_kv - 1
+    // query tile i uses the unit's KV tiles lo[i] .. hi[i] - 1 (relative to kv0); lo = hi: none
+    // (no row inside the sequence, or no row with a key in reach)
+    int lo[2], hi[2];
     bool skip;
 };
 
-template <int ROWS, int BK>
+// LOCAL: the window has a bounded left side, so query tiles may start past KV tile 0.
+// Without it kv0 and lo[] are 0 and the accessors below fold them away.
+template <int ROWS, int BK, bool LOCAL>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     Unit t;
     const int per_m = p.num_seqs * p.Hq;
@@ -76,8 +84,9 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
         // malformed offsets can only shrink the work: rows are clipped to the tensors
         t.q_start = max(t.q_start, 0);
         t.k_start = max(t.k_start, 0);
-        t.Lq = max(min(t.Lq, p.Tq - t.q_start), 0);
-        t.Lk = max(min(t.Lk, p.Tk - t.k_start), 0);
+        // (and to 2^30 tokens, the longest sequence the window arithmetic below is exact for)
+        t.Lq = max(min(min(t.Lq, p.Tq - t.q_start), 1 << 30), 0);
+        t.Lk = max(min(min(t.Lk, p.Tk - t.k_start), 1 << 30), 0);
     } else {
         t.q_start = t.b * p.Sq;
         t.Lq = p.Sq;
@@ -86,18 +95,64 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     }
     t.q0 = m * ROWS;
     t.skip = t.q0 >= t.Lq;
-    t.n_kv = 0;
+    t.kv0 = 0;
+    t.lo[0] = t.lo[1] = 0;
+    if constexpr (!LOCAL) {
+        // every query tile starts at KV tile 0 and stops after the last tile its rows can see
+        t.n_kv = 0;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            const int row_begin = t.q0 + 128 * i;              // query tiles are 128 rows
+            const int row_end = min(row_begin + 128, t.Lq);   // exclusive
+            int kend = row_end > row_begin ? t.Lk : 0;
+            if (p.wr >= 0 && row_end > row_begin) kend = min(kend, row_end + (t.Lk - t.Lq) + p.wr);
+            t.hi[i] = kend > 0 ? (kend + BK - 1) / BK : 0;
+            if (i * 128 < ROWS) t.n_kv = max(t.n_kv, t.hi[i]);
+            else t.hi[i] = 0;
+        }
+        return t;
+    }
+    int f[2], e[2], kmin = 0x7fffffff, kmax = 0;
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-        const int row_begin = t.q0 + 128 * i;              // query tiles are 128 rows
-        const int row_end = min(row_begin + 128, t.Lq);   // exclusive
-        int kend = row_end > row_begin ? t.Lk : 0;
-        if (p.causal && row_end > row_begin) kend = min(kend, row_end - 1 + (t.Lk - t.Lq) + 1);
-        t.n_tile[i] = kend > 0 ? (kend + BK - 1) / BK : 0;
-        if (i * 128 < ROWS) t.n_kv = max(t.n_kv, t.n_tile[i]);
-        else t.n_tile[i] = 0;
+        const int row_begin = t.q0 + 128 * i;
+        const int row_end = min(row_begin + 128, t.Lq);
+        f[i] = e[i] = 0;
+        if (i * 128 < ROWS && row_end > row_begin) {
+            // keys reachable from rows row_begin .. row_end-1 (lengths <= 2^30 and window sides < 2^30
+            // keep every term inside int32)
+            const int off = t.Lk - t.Lq;
+            const int lo = max(0, row_begin + off - p.wl);
+            int hi = t.Lk - 1;
+            if (p.wr >= 0) hi = min(hi, row_end - 1 + off + p.wr);
+            if (hi >= lo) {
+                f[i] = lo / BK;
+                e[i] = hi / BK + 1;
+                kmin = min(kmin, f[i]);
+                kmax = max(kmax, e[i]);
+            }
+        }
+    }
+    t.kv0 = kmax > 0 ? kmin : 0;
+    t.n_kv = kmax > 0 ? kmax - kmin : 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        t.lo[i] = e[i] > 0 ? f[i] - t.kv0 : 0;
+        t.hi[i] = e[i] > 0 ? e[i] - t.kv0 : 0;
     }
     return t;
+}
+
+template <bool LOCAL>
+__device__ __forceinline__ int unit_lo(const Unit& t, int i) {
+    if constexpr (LOCAL) return i == 0 ? t.lo[0] : t.lo[1];
+    else return 0;
+}
+__device__ __forceinline__ int unit_hi(const Unit& t, int i) { return i == 0 ? t.hi[0] : t.hi[1]; }
+template <bool LOCAL>
+__device__ __forceinline__ int unit_kv0(const Unit& t) {
+    if constexpr (LOCAL) return t.kv0;
+    else return 0;
 }
 
 template <int D, int NQ, int BK, int KST>
@@ -129,7 +184,7 @@ constexpr float kDeferLog2 = 8.0f;
 constexpr int kFmaExpEvery = 0;
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D, int NQ, int BK, int KST>
+template <int D, int NQ, int BK, int KST, bool LOCAL>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
@@ -197,7 +252,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             uint32_t kv_it = 0, q_it = 0;
             for (int k = 0, u = snake_unit(0, p.num_units); u >= 0; u = snake_unit(++k, p.num_units)) {
                 if (u >= p.num_units) continue;
-                const Unit t = decode_unit<ROWS, BK>(p, u);
+                const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
                 if (t.skip || t.n_kv == 0) continue;
                 const int hk = t.h / p.group;
                 bool ok = true;
@@ -220,13 +275,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c)
                         tma_load_3d(smem_u32(sK + st * C::KV_BYTES + c * BK * 128), &tmK, k_full(st), c * 64, hk,
-                                    t.k_start + j * BK);
+                                    t.k_start + (unit_kv0<LOCAL>(t) + j) * BK);
                     if (n > 0 && !mbar_wait(v_empty(st), (n - 1) & 1, w)) { ok = false; break; }
                     mbar_arrive_expect_tx(v_full(st), C::KV_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c)
                         tma_load_3d(smem_u32(sV + st * C::KV_BYTES + c * BK * 128), &tmV, v_full(st), c * 64, hk,
-                                    t.k_start + j * BK);
+                                    t.k_start + (unit_kv0<LOCAL>(t) + j) * BK);
                 }
                 if (!ok) break;
             }
@@ -257,7 +312,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             bool ok = true;
             for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
                 if (u >= p.num_units) continue;
-                const Unit t = decode_unit<ROWS, BK>(p, u);
+                const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
                 if (t.skip || t.n_kv == 0) continue;
                 for (int i = 0; i < NQ && ok; ++i)
                     if (!mbar_wait(q_full(i), q_it & 1, w)) ok = false;
@@ -268,7 +323,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     if (!mbar_wait(k_full(st), (kv_it / KST) & 1, w)) break;
                     tc_fence_after();
                     for (int i = 0; i < NQ; ++i) {
-                        if (t.n_tile[i] == 0) continue;
+                        if (unit_lo<LOCAL>(t, i) != 0 || unit_hi(t, i) == 0) continue;   // tile i starts later (or never)
                         issue_qk(i, st);
                         umma_commit(s_full(i));
                     }
@@ -276,7 +331,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     if (t.n_kv == 1)
                         for (int i = 0; i < NQ; ++i) umma_commit(q_empty(i));
                 }
-                // query tile i stops after its own last visible KV tile (n_tile[i] <= n_kv)
+                // query tile i works on the unit's KV tiles lo[i] .. hi[i]-1
                 for (int j = 0; j < t.n_kv && ok; ++j) {
                     const uint32_t cur = kv_it + j;
                     const int st = cur % KST;
@@ -286,14 +341,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     tc_fence_after();
                     bool k_ready = false;
                     for (int i = 0; i < NQ; ++i) {
-                        if (j < t.n_tile[i]) {
+                        if (j >= unit_lo<LOCAL>(t, i) && j < unit_hi(t, i)) {
                             if (!mbar_wait(p_full(i), p_it[i] & 1, w)) { ok = false; break; }
                             ++p_it[i];
                             tc_fence_after();
-                            issue_pv(i, st, j > 0);
+                            issue_pv(i, st, j > unit_lo<LOCAL>(t, i));
                             umma_commit(o_full(i));
                         }
-                        if (j + 1 < t.n_tile[i]) {
+                        if (j + 1 >= unit_lo<LOCAL>(t, i) && j + 1 < unit_hi(t, i)) {
                             if (!k_ready) {
                                 if (!mbar_wait(k_full(stn), (nxt / KST) & 1, w)) { ok = false; break; }
                                 tc_fence_after();
@@ -304,6 +359,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                         }
                     }
                     if (!ok) break;
+                    // K(j+1) was waited for above whenever j+1 < n_kv: the two query tiles' ranges
+                    // overlap or touch (the first key row of tile 1 is at most one past the last key
+                    // row of tile 0, since the window sides are >= 0), so their union has no gap
+                    // and some tile issues QK(j+1)
                     umma_commit(v_empty(st));
                     if (j + 1 < t.n_kv) {
                         umma_commit(k_empty(stn));
@@ -330,13 +389,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
         bool ok = true;
         for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
             if (u >= p.num_units) continue;
-            const Unit t = decode_unit<ROWS, BK>(p, u);
+            const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
             if (t.skip) continue;
             const int row = t.q0 + i * BM + r;
             const bool valid = row < t.Lq;
             __nv_bfloat16* orow = p.o + (static_cast<size_t>(t.q_start + row) * p.Hq + t.h) * D;
             float* lse_ptr = p.lse + t.b * p.lse_sB + t.h * p.lse_sH + static_cast<long long>(t.q_start) * p.lse_sT + row;
-            const int n_mine = t.n_tile[i];          // KV tiles this query tile sees
+            const int lo_i = unit_lo<LOCAL>(t, i);
+            const int n_mine = unit_hi(t, i) - lo_i;       // KV tiles this query tile sees
             if (n_mine == 0) {
                 if (valid) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
@@ -345,8 +405,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                 }
                 continue;
             }
-            const int off = t.Lk - t.Lq;
-            const int key_lim = p.causal ? min(t.Lk - 1, row + off) : (t.Lk - 1);
+            // keys key_lo .. key_hi of the sequence are allowed for this row
+            int key_lo = 0, key_hi = t.Lk - 1;
+            if (LOCAL) key_lo = max(0, row + (t.Lk - t.Lq) - p.wl);
+            if (p.wr >= 0) key_hi = min(key_hi, row + (t.Lk - t.Lq) + p.wr);
             float m_ref = -INFINITY;
             float l = 0.f;
             for (int j = 0; j < n_mine; ++j) {
@@ -364,10 +426,11 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
 #pragma unroll
                     for (int cc = 1; cc < BK / 32; ++cc) reg_tie(*reinterpret_cast<uint32_t(*)[32]>(sr + cc * 32));
                 }
-                const int kbase = j * BK;
-                if (__any_sync(0xffffffffu, kbase + BK - 1 > key_lim)) {
+                const int kbase = (unit_kv0<LOCAL>(t) + lo_i + j) * BK;
+                if (__any_sync(0xffffffffu, kbase + BK - 1 > key_hi || (LOCAL && kbase < key_lo))) {
 #pragma unroll
-                    for (int c = 0; c < BK; ++c) s[c] = (kbase + c <= key_lim) ? s[c] : -INFINITY;
+                    for (int c = 0; c < BK; ++c)
+                        s[c] = (kbase + c <= key_hi && (!LOCAL || kbase + c >= key_lo)) ? s[c] : -INFINITY;
                 }
                 float mx[4] = {s[0], s[1], s[2], s[3]};
 #pragma unroll
@@ -475,7 +538,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     }
 }
 
-template <int D, int NQ, int BK, int KST>
+template <int D, int NQ, int BK, int KST, bool LOCAL>
 static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream) {
     using C = FwdCfg<D, NQ, BK, KST>;
     alignas(64) CUtensorMap mq, mk, mv;
@@ -502,7 +565,8 @@ static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, 
     if (units > 0x7fffffffLL) return 2;
     p.num_units = static_cast<int>(units);
     p.scale_log2 = pr.scale * 1.4426950408889634f;
-    p.causal = pr.causal;
+    p.wl = pr.wl;
+    p.wr = pr.wr;
     p.lse_sB = pr.lse_sB;
     p.lse_sH = pr.lse_sH;
     p.lse_sT = pr.lse_sT;
@@ -510,7 +574,7 @@ static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, 
     p.status = dev.status;
     if (p.num_units == 0) return 0;
 
-    auto kern = fwd_kernel<D, NQ, BK, KST>;
+    auto kern = fwd_kernel<D, NQ, BK, KST, LOCAL>;
     static bool attr_set[64] = {};
     if (!attr_set[dev.id & 63]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
@@ -532,10 +596,14 @@ static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, 
 }
 
 int launch_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream) {
+    const bool local = pr.wl >= 0;
     switch (pr.D) {
-        case 64: return run_fwd<64, 2, 128, 4>(pr, out, lse, dev, stream);
-        case 128: return run_fwd<128, 2, 128, 2>(pr, out, lse, dev, stream);
-        case 256: return run_fwd<256, 1, 128, 1>(pr, out, lse, dev, stream);
+        case 64: return local ? run_fwd<64, 2, 128, 4, true>(pr, out, lse, dev, stream)
+                              : run_fwd<64, 2, 128, 4, false>(pr, out, lse, dev, stream);
+        case 128: return local ? run_fwd<128, 2, 128, 2, true>(pr, out, lse, dev, stream)
+                               : run_fwd<128, 2, 128, 2, false>(pr, out, lse, dev, stream);
+        case 256: return local ? run_fwd<256, 1, 128, 1, true>(pr, out, lse, dev, stream)
+                               : run_fwd<256, 1, 128, 1, false>(pr, out, lse, dev, stream);
         default: return 2;
     }
 }

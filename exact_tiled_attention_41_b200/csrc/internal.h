@@ -22,7 +22,10 @@ struct Problem {
     int Tq, Tk;          // total tokens
     int Hq, Hkv, D;
     float scale;
-    int causal;
+    // Sliding window (README, flash_attn_func docstring): query i keeps the keys j with
+    // i + Lk - Lq - wl <= j <= i + Lk - Lq + wr; -1 leaves that side unbounded.
+    // A causal mask is wr = 0 (with or without a window on the left).
+    int wl, wr;
     // LSE addressing: index = b * lse_sB + h * lse_sH + tok_start * lse_sT + row
     long long lse_sB, lse_sH;
     int lse_sT;
@@ -47,8 +50,9 @@ size_t bwd_workspace_bytes(long long Tq, int Hq, int D);
 // head dim 256: main backward kernel + dQ convert (after the shared preprocess)
 int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,
                        void* dq, void* dk, void* dv, const Device& dev, cudaStream_t stream);
+// deterministic: dQ from a separate query-tile-stationary pass instead of float32 reduce-adds
 int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
-               void* dv, void* workspace, const Device& dev, cudaStream_t stream);
+               void* dv, void* workspace, bool deterministic, const Device& dev, cudaStream_t stream);
 
 struct Decode {
     const void* q;            // [B, 1, Hq, D]

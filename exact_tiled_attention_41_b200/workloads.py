@@ -30,6 +30,7 @@ class Workload:
     scale: float
     tensors: dict = field(default_factory=dict)
     meta: dict = field(default_factory=dict)
+    window: tuple = (-1, -1)       # sliding window (left, right); -1 = unbounded side
 
 
 def _randn(g, shape):

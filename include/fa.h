@@ -132,6 +132,50 @@ FA_API int fa_varlen_bwd(const void* q, const void* k, const void* v, const void
                   int Hq, int Hkv, int D, float softmax_scale, int causal,
                   void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
+/* ------------------------------------------------------------------------- sliding window, deterministic backward
+ * The *_ex entry points are the four calls above with the remaining options of
+ * flash_attn_func / flash_attn_varlen_func (README, flash_attn_func docstring);
+ * the calls above are the *_ex calls with window_left = window_right = -1 and
+ * deterministic = 0.  Workspace needs and sizes are those of the plain calls.
+ *
+ * window_left, window_right: sliding window local attention (README changelog
+ *   2.3, flash_attn_func docstring).  Query i of a sequence keeps only the keys
+ *   j with  i + Sk - Sq - window_left <= j <= i + Sk - Sq + window_right
+ *   (bottom-right aligned like the causal mask; Sq, Sk the lengths of that
+ *   sequence).  A negative side (-1) is unbounded; (-1, -1) is no window.  With
+ *   causal != 0 the keys kept are those both rules keep, i.e. the right side is
+ *   0.  Rows left with no key give out = 0, lse = -inf and zero gradients.
+ * deterministic (backward only): 0 accumulates dq with float32 reduce-adds whose
+ *   order varies from run to run; 1 computes dq in a separate pass in which each
+ *   query tile sums its key tiles in a fixed order, so dq, dk and dv are
+ *   bit-identical across runs on the same inputs (README: the deterministic
+ *   backward is slightly slower; the forward is always deterministic).
+ * Errors as for the plain calls; sequence lengths above 2^30 are
+ * FA_ERR_UNSUPPORTED on every dense and varlen entry point.
+ */
+FA_API int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                     float softmax_scale, int causal, int window_left, int window_right,
+                     void* workspace, size_t workspace_bytes, fa_stream_t stream);
+FA_API int fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                     const float* lse, void* dq, void* dk, void* dv,
+                     int B, int Hq, int Hkv, int Sq, int Sk, int D,
+                     float softmax_scale, int causal, int window_left, int window_right, int deterministic,
+                     void* workspace, size_t workspace_bytes, fa_stream_t stream);
+FA_API int fa_varlen_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                            int Hq, int Hkv, int D, float softmax_scale, int causal,
+                            int window_left, int window_right,
+                            void* workspace, size_t workspace_bytes, fa_stream_t stream);
+FA_API int fa_varlen_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                            const float* lse, void* dq, void* dk, void* dv,
+                            const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k,
+                            int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                            int Hq, int Hkv, int D, float softmax_scale, int causal,
+                            int window_left, int window_right, int deterministic,
+                            void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
 /* ------------------------------------------------------------------------- KV-cache decode
  * fa_fwd_kvcache: new queries against a contiguous KV cache (README,
  * flash_attn_with_kvcache docstring; changelog 2.2: the cache load is split

@@ -52,47 +52,48 @@ def check_grad(x_gpu, ref, name, tol=GRAD_TOL):
     return e
 
 
-def run_dense(w, backward=True):
+def run_dense(w, backward=True, deterministic=False):
     t = w.tensors
     q, k, v = t["q"].cuda(), t["k"].cuda(), t["v"].cuda()
-    out, lse = A.flash_attn_func(q, k, v, w.scale, w.causal)
+    out, lse = A.flash_attn_func(q, k, v, w.scale, w.causal, w.window)
     res = dict(out=out, lse=lse)
     if backward:
         do = t["do"].cuda()
-        res["dq"], res["dk"], res["dv"] = A.flash_attn_backward(do, q, k, v, out, lse, w.scale, w.causal)
+        res["dq"], res["dk"], res["dv"] = A.flash_attn_backward(do, q, k, v, out, lse, w.scale, w.causal, w.window,
+                                                                deterministic)
     torch.cuda.synchronize()
     return res
 
 
-def check_dense(w, backward=True):
-    res = run_dense(w, backward)
+def check_dense(w, backward=True, deterministic=False):
+    res = run_dense(w, backward, deterministic)
     t = w.tensors
     qn, kn, vn = f64(t["q"]), f64(t["k"]), f64(t["v"])
-    o_ref, l_ref = oracle.mha_forward(qn, kn, vn, w.scale, w.causal)
+    o_ref, l_ref = oracle.mha_forward(qn, kn, vn, w.scale, w.causal, w.window)
     errs = dict(o=check_o(res["out"], o_ref), lse=check_lse(res["lse"], l_ref))
     if backward:
-        dq, dk, dv = oracle.mha_backward(qn, kn, vn, f64(t["do"]), w.scale, w.causal)
+        dq, dk, dv = oracle.mha_backward(qn, kn, vn, f64(t["do"]), w.scale, w.causal, w.window)
         errs["dq"] = check_grad(res["dq"], dq, "dQ")
         errs["dk"] = check_grad(res["dk"], dk, "dK")
         errs["dv"] = check_grad(res["dv"], dv, "dV")
     return errs
 
 
-def check_varlen(w, backward=True):
+def check_varlen(w, backward=True, deterministic=False):
     t = w.tensors
     m = w.meta
     q, k, v = t["q"].cuda(), t["k"].cuda(), t["v"].cuda()
     cq, ck = t["cu_q"].cuda(), t["cu_k"].cuda()
-    out, lse = A.flash_attn_varlen_func(q, k, v, cq, ck, m["max_q"], m["max_k"], w.scale, w.causal)
+    out, lse = A.flash_attn_varlen_func(q, k, v, cq, ck, m["max_q"], m["max_k"], w.scale, w.causal, w.window)
     qn, kn, vn = f64(t["q"]), f64(t["k"]), f64(t["v"])
     cu_q, cu_k = t["cu_q"].numpy(), t["cu_k"].numpy()
-    o_ref, l_ref = oracle.varlen_forward(qn, kn, vn, cu_q, cu_k, w.scale, w.causal)
+    o_ref, l_ref = oracle.varlen_forward(qn, kn, vn, cu_q, cu_k, w.scale, w.causal, w.window)
     errs = dict(o=check_o(out, o_ref), lse=check_lse(lse, l_ref))
     if backward:
         do = t["do"].cuda()
         dq, dk, dv = A.flash_attn_varlen_backward(do, q, k, v, out, lse, cq, ck, m["max_q"], m["max_k"], w.scale,
-                                                  w.causal)
-        rq, rk, rv = oracle.varlen_backward(qn, kn, vn, f64(t["do"]), cu_q, cu_k, w.scale, w.causal)
+                                                  w.causal, w.window, deterministic)
+        rq, rk, rv = oracle.varlen_backward(qn, kn, vn, f64(t["do"]), cu_q, cu_k, w.scale, w.causal, w.window)
         errs["dq"] = check_grad(dq, rq, "dQ")
         errs["dk"] = check_grad(dk, rk, "dK")
         errs["dv"] = check_grad(dv, rv, "dV")
