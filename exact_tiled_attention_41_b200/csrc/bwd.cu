@@ -33,6 +33,9 @@
 //                    bf16 P^T / dS^T, so the dQ read-out overlaps   (N-major x N-major)
 //                    dV += P^T dO, dK += dS^T Q               (tensor-memory A)
 //   3. convert: dQ = bf16(scale * dQacc).
+// The deterministic backward runs the main kernel with DQ = false (no dQ product,
+// no reduce-adds, warps 8-11 idle) and computes dq in the query-tile-stationary
+// pass of bwd_dq.cu instead of steps 2's dQ and 3.
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -128,7 +131,7 @@ struct BwdCfg {
     static_assert(2 * 128 * COMPUTE_REGS + 128 * DQ_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
-template <int D>
+template <int D, bool DQ>
 __global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -256,7 +259,7 @@ __global__ void __launch_bounds__(512, 1)
                     for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
                         const int st = q_it % ST;
                         if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
-                        if (g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
+                        if (DQ && g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
                         tc_fence_after();
                         const uint8_t* sq = smem + C::OFF_Q + st * C::T_BYTES;
                         const uint8_t* sdo = smem + C::OFF_DO + st * C::T_BYTES;
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(512, 1)
                                     sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
                         }
                         // the previous tile's dQ columns in the dP^T region must be read out first
-                        if (g_it > 0 && !mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
+                        if (DQ && g_it > 0 && !mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
@@ -278,19 +281,21 @@ __global__ void __launch_bounds__(512, 1)
                         umma_commit(s_full);
                         if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
-                        // dQ = dS K first, into the free high columns, so its read-out overlaps dV / dK
+                        if constexpr (DQ) {
+                            // dQ = dS K first, into the free high columns, so its read-out overlaps dV / dK
 #pragma unroll
-                        for (int hh = 0; hh < D / 64; ++hh) {
+                            for (int hh = 0; hh < D / 64; ++hh) {
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
-                                umma_ss(tmem + C::COL_DQ(hh),
-                                        sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
-                                        sdesc_sw128(smem_u32(smem + C::OFF_K + hh * 128 * 128 + kk * 16 * 128),
-                                                    128 * 128, 1024),
-                                        id_dq, kk > 0);
+                                for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
+                                    umma_ss(tmem + C::COL_DQ(hh),
+                                            sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
+                                            sdesc_sw128(smem_u32(smem + C::OFF_K + hh * 128 * 128 + kk * 16 * 128),
+                                                        128 * 128, 1024),
+                                            id_dq, kk > 0);
+                                }
                             }
+                            umma_commit(dq_full);
                         }
-                        umma_commit(dq_full);
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 query rows
                             const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
@@ -312,6 +317,7 @@ __global__ void __launch_bounds__(512, 1)
     } else if (warp >= 8) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::DQ_REGS));
         // ------------------------------------------------------------ dQ warpgroup (thread = query row)
+        if constexpr (DQ) {
         const int wq = warp - 8;
         const int r = wq * 32 + lane;
         const uint32_t lb = tmem_lane_base(wq);
@@ -351,6 +357,7 @@ __global__ void __launch_bounds__(512, 1)
                     }
                 }
             }
+        }
         }
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
@@ -503,7 +510,7 @@ __global__ void __launch_bounds__(512, 1)
 
 // ---------------------------------------------------------------------------- preprocess
 // One warp per (query token, head): Delta = sum_d dO * O (fp32), LSE2 = LSE * log2(e)
-// (+inf where LSE = -inf).  Also zeroes the dQ accumulator (grid-stride).
+// (+inf where LSE = -inf).  Also zeroes the dQ accumulator (grid-stride) unless dq_acc is NULL.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
                                                       const float* lse, float* lse2, float* delta, float* dq_acc,
@@ -512,7 +519,7 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
     const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     const long long rows = static_cast<long long>(Tq) * Hq;
-    {
+    if (dq_acc != nullptr) {
         const long long n4 = rows * D / 4;
         float4* z = reinterpret_cast<float4*>(dq_acc);
         for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
@@ -593,7 +600,7 @@ size_t bwd_workspace_bytes(long long Tq, int Hq, int D) {
     return up(acc) + 2 * up(stat);
 }
 
-template <int D>
+template <int D, bool DQ>
 static int run_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk, void* dv,
                    void* workspace, const Device& dev, cudaStream_t stream) {
     using C = BwdCfg<D>;
@@ -608,8 +615,8 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
         const long long cap = static_cast<long long>(dev.num_sms) * 16;
         if (blocks > cap) blocks = cap;
         bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
-            static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta, dq_acc,
-            pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+            static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
+            DQ ? dq_acc : nullptr, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
 
@@ -647,7 +654,7 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
 
-    auto kern = bwd_kernel<D>;
+    auto kern = bwd_kernel<D, DQ>;
     static bool set[64] = {};
     if (!set[dev.id & 63]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
@@ -665,6 +672,7 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
         prof_after(1, stream);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
+    if (!DQ) return launch_bwd_dq(pr, dout, lse2, delta, dq, dev, stream);
     dim3 cg((pr.Tq + 31) / 32, pr.Hq);
     bwd_convert_kernel<D><<<cg, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), pr.Tq, pr.Hq, pr.scale);
     return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
@@ -672,7 +680,7 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
 
 // Head dim 256: same preprocess, then the half-head-dim kernel of bwd256.cu (which also converts dQ).
 static int run_bwd256(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
-                      void* dv, void* workspace, const Device& dev, cudaStream_t stream) {
+                      void* dv, void* workspace, bool det, const Device& dev, cudaStream_t stream) {
     constexpr int D = 256;
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     float* dq_acc = static_cast<float*>(workspace);
@@ -683,19 +691,24 @@ static int run_bwd256(const Problem& pr, const void* out, const void* dout, cons
     const long long cap = static_cast<long long>(dev.num_sms) * 16;
     if (blocks > cap) blocks = cap;
     bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta, dq_acc,
-        pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+        static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
+        det ? nullptr : dq_acc, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
     if (cudaPeekAtLastError() != cudaSuccess) return 5;
-    return launch_bwd256_main(pr, dout, lse2, delta, dq_acc, dq, dk, dv, dev, stream);
+    const int st = launch_bwd256_main(pr, dout, lse2, delta, dq_acc, dq, dk, dv, !det, dev, stream);
+    if (st != 0 || !det) return st;
+    return launch_bwd_dq(pr, dout, lse2, delta, dq, dev, stream);
 }
 
 int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk, void* dv,
                void* workspace, bool deterministic, const Device& dev, cudaStream_t stream) {
-    if (deterministic) return 2;
     switch (pr.D) {
-        case 64: return run_bwd<64>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
-        case 128: return run_bwd<128>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
-        case 256: return run_bwd256(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
+        case 64:
+            return deterministic ? run_bwd<64, false>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream)
+                                 : run_bwd<64, true>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
+        case 128:
+            return deterministic ? run_bwd<128, false>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream)
+                                 : run_bwd<128, true>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
+        case 256: return run_bwd256(pr, out, dout, lse, dq, dk, dv, workspace, deterministic, dev, stream);
         default: return 2;
     }
 }

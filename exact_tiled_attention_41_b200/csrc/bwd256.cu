@@ -15,6 +15,8 @@
 //   accumulator is laid out [Hq][Tq][256].
 // Roles: warps 0-3 compute (thread = key row), 4-7 dQ (thread = head-dim row),
 // 8 producer, 9 MMA issuer, 10-11 idle; registers redistributed with setmaxnreg.
+// With DQ = false (the deterministic backward) dQ is left to the query-tile-stationary
+// pass of bwd_dq.cu: no dQ product, no reduce-adds, no convert.
 #include "internal.h"
 #include "sm100.cuh"
 
@@ -99,6 +101,7 @@ struct Cfg {
     static_assert(128 * COMPUTE_REGS + 2 * 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
+template <bool DQ>
 __global__ void __launch_bounds__(384, 1)
     bwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -230,18 +233,20 @@ __global__ void __launch_bounds__(384, 1)
                         }
                         umma_commit(s_full);
                         if (!mbar_wait(p_full, q_it & 1, w)) { ok = false; break; }
-                        if (q_it > 0 && !mbar_wait(dq_empty, (q_it - 1) & 1, w)) { ok = false; break; }
+                        if (DQ && q_it > 0 && !mbar_wait(dq_empty, (q_it - 1) & 1, w)) { ok = false; break; }
                         tc_fence_after();
-                        // dQ^T half = K[:, half]^T dS^T (K-dim = 128 keys)
+                        if constexpr (DQ) {
+                            // dQ^T half = K[:, half]^T dS^T (K-dim = 128 keys)
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            umma_ss(tmem + C::COL_DQ,
-                                    sdesc_sw128(smem_u32(smem + C::OFF_K + 2 * t.hh * 128 * 128 + kk * 16 * 128),
-                                                128 * 128, 1024),
-                                    sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024), id_q,
-                                    kk > 0);
+                            for (int kk = 0; kk < 8; ++kk) {
+                                umma_ss(tmem + C::COL_DQ,
+                                        sdesc_sw128(smem_u32(smem + C::OFF_K + 2 * t.hh * 128 * 128 + kk * 16 * 128),
+                                                    128 * 128, 1024),
+                                        sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
+                                        id_q, kk > 0);
+                            }
+                            umma_commit(dq_full);
                         }
-                        umma_commit(dq_full);
                         // dV half += P^T dO[:, half], dK half += dS^T Q[:, half] (K-dim = 64 queries)
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
@@ -264,7 +269,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             __syncwarp();
-        } else if (warp < 8) {
+        } else if (DQ && warp < 8) {
             // -------------------------------------------------------- dQ warpgroup (thread = head-dim row)
             const int wq = warp - 4;
             const int r = wq * 32 + lane;
@@ -440,8 +445,9 @@ __global__ void __launch_bounds__(256) bwd256_convert_kernel(const float* dq_acc
 
 }  // namespace
 
-int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,
-                       void* dq, void* dk, void* dv, const Device& dev, cudaStream_t stream) {
+template <bool DQ>
+static int run_bwd256(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,
+                      void* dq, void* dk, void* dv, const Device& dev, cudaStream_t stream) {
     using C = Cfg;
     alignas(64) CUtensorMap mq, mk, mv, mdo;
     const uint64_t rq = static_cast<uint64_t>(pr.Hq) * D * 2, rk = static_cast<uint64_t>(pr.Hkv) * D * 2;
@@ -474,29 +480,36 @@ int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, c
     p.wr = pr.wr;
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
+    auto kern = bwd256_kernel<DQ>;
     static bool set[64] = {};
     if (!set[dev.id & 63]) {
-        if (cudaFuncSetAttribute(bwd256_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(C::SMEM)) != cudaSuccess)
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
+            cudaSuccess)
             return 5;
         cudaFuncAttributes fa_attr;
-        if (cudaFuncGetAttributes(&fa_attr, bwd256_kernel) != cudaSuccess || fa_attr.numRegs != C::LAUNCH_REGS)
-            return 2;
+        if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess || fa_attr.numRegs != C::LAUNCH_REGS) return 2;
         set[dev.id & 63] = true;
     }
     const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
     if (grid > 0) {
         prof_before(1, stream);
-        bwd256_kernel<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
         prof_after(1, stream);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
+    if (!DQ) return 0;
     const long long n2 = static_cast<long long>(pr.Tq) * pr.Hq * (D / 2);
     long long blocks = (n2 + 255) / 256;
     if (blocks > static_cast<long long>(dev.num_sms) * 32) blocks = static_cast<long long>(dev.num_sms) * 32;
     bwd256_convert_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), pr.Tq,
                                                                         pr.Hq, pr.scale);
     return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
+}
+
+int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,
+                       void* dq, void* dk, void* dv, bool with_dq, const Device& dev, cudaStream_t stream) {
+    return with_dq ? run_bwd256<true>(pr, dout, lse2, delta, dq_acc, dq, dk, dv, dev, stream)
+                   : run_bwd256<false>(pr, dout, lse2, delta, dq_acc, dq, dk, dv, dev, stream);
 }
 
 }  // namespace fa

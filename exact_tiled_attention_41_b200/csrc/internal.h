@@ -47,9 +47,13 @@ void prof_after(int kernel_id, cudaStream_t s);
 int launch_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream);
 
 size_t bwd_workspace_bytes(long long Tq, int Hq, int D);
-// head dim 256: main backward kernel + dQ convert (after the shared preprocess)
+// head dim 256: main backward kernel + dQ convert (after the shared preprocess); with_dq = false
+// leaves dq alone (the deterministic backward computes it with launch_bwd_dq)
 int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,
-                       void* dq, void* dk, void* dv, const Device& dev, cudaStream_t stream);
+                       void* dq, void* dk, void* dv, bool with_dq, const Device& dev, cudaStream_t stream);
+// deterministic dQ: query-tile-stationary pass writing bf16 dq from LSE2 / Delta of the preprocess
+int launch_bwd_dq(const Problem& pr, const void* dout, const float* lse2, const float* delta, void* dq,
+                  const Device& dev, cudaStream_t stream);
 // deterministic: dQ from a separate query-tile-stationary pass instead of float32 reduce-adds
 int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
                void* dv, void* workspace, bool deterministic, const Device& dev, cudaStream_t stream);

@@ -87,6 +87,28 @@ def test_bwd_checks_workspace_before_launch(lib):
     assert st == abi.FA_ERR_INVALID_ARG
 
 
+def test_ex_entry_points_validate_like_the_plain_calls(lib):
+    # window sides and the deterministic flag never make a bad call valid
+    st = abi.fa_fwd_ex(None, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, 128, 128, 128, 0.1, 1, 64, -1, stream=S0)
+    assert st == abi.FA_ERR_INVALID_ARG
+    st = abi.fa_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 3, 2, 128, 128, 128, 0.1, 0, 5, 5, stream=S0)
+    assert st == abi.FA_ERR_INVALID_ARG
+    st = abi.fa_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, 1, 4, 2, (1 << 30) + 1, 128, 128, 0.1, 0, -1, -1, stream=S0)
+    assert st == abi.FA_ERR_UNSUPPORTED          # sequences are limited to 2^30 tokens
+    need = abi.fa_bwd_workspace_size(2, 4, 2, 300, 300, 128)
+    for det in (0, 1):
+        st = abi.fa_bwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 300, 300, 128, 0.1, 1,
+                           32, -1, det, FAKE, need - 1, S0)
+        assert st == abi.FA_ERR_WORKSPACE
+    st = abi.fa_varlen_fwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 2, 10, 10, 20, 20, 2, 2, 64, 0.1, 1, 4, 0,
+                              stream=S0)
+    assert st == abi.FA_ERR_INVALID_ARG
+    nv = abi.fa_varlen_bwd_workspace_size(2, 20, 20, 2, 2, 64)
+    st = abi.fa_varlen_bwd_ex(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 10, 20, 20,
+                              2, 2, 64, 0.1, 1, 4, 0, 1, FAKE + 16, nv, S0)
+    assert st == abi.FA_ERR_ALIGNMENT
+
+
 def test_varlen_rejects_missing_cu_seqlens(lib):
     st = abi.fa_varlen_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 2, 10, 10, 20, 20, 2, 2, 64, 0.1, 1, stream=S0)
     assert st == abi.FA_ERR_INVALID_ARG
