@@ -42,6 +42,17 @@ def fwd_flops(B, H, Sq, Sk, D, causal):
     return 4.0 * B * H * Sq * Sk * D * (0.5 if causal else 1.0)
 
 
+def window_pairs(Sq, Sk, left, right, causal):
+    """Number of (query, key) pairs a bottom-right aligned window (and causal mask) keeps."""
+    import numpy as np
+    i = np.arange(Sq, dtype=np.int64)
+    off = Sk - Sq
+    lo = np.zeros(Sq, dtype=np.int64) if left < 0 else np.maximum(i + off - left, 0)
+    r = 0 if causal else right
+    hi = np.full(Sq, Sk - 1, dtype=np.int64) if (r < 0 and not causal) else np.minimum(i + off + max(r, 0), Sk - 1)
+    return int(np.maximum(hi - lo + 1, 0).sum())
+
+
 def max_over_ranks(value, world, device="cpu"):
     """The slowest rank's figure; every rank takes part in the same collective (no-op for one rank)."""
     if world <= 1:
@@ -381,10 +392,24 @@ def measure_extras(torch, abi, A, W, dev, pk):
                                    stream), 5)
     bms = timed(lambda: abi.fa_bwd(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, B, Hq, Hkv, S, S, D,
                                    w.scale, 1, ws, nb, stream), 3)
+    # the same backward with deterministic dq (query-tile-stationary pass, fixed summation order)
+    dms = timed(lambda: abi.fa_bwd_ex(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, B, Hq, Hkv, S, S, D,
+                                      w.scale, 1, -1, -1, 1, ws, nb, stream), 3)
     res["gqa_long_B2_Hq32_Hkv8_S8192_D128_causal"] = {
         "fwd_ms": fms, "fwd_tflops": ff / fms / 1e9, "bwd_ms": bms, "bwd_tflops": 2.5 * ff / bms / 1e9,
         "fwd_frac_of_measured_peak": ff / fms / 1e9 / pk["bf16_tflops"],
-        "bwd_frac_of_measured_peak": 2.5 * ff / bms / 1e9 / pk["bf16_tflops"]}
+        "bwd_frac_of_measured_peak": 2.5 * ff / bms / 1e9 / pk["bf16_tflops"],
+        "bwd_deterministic_ms": dms, "bwd_deterministic_tflops": 2.5 * ff / dms / 1e9}
+    # sliding window of 4096 keys (causal): FLOPs of the pairs the window keeps
+    wf = 4.0 * B * Hq * D * window_pairs(S, S, 4096, 0, True)
+    wfms = timed(lambda: abi.fa_fwd_ex(t["q"], t["k"], t["v"], out, lse, B, Hq, Hkv, S, S, D, w.scale, 1, 4096, 0,
+                                       None, 0, stream), 5)
+    wbms = timed(lambda: abi.fa_bwd_ex(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, B, Hq, Hkv, S, S, D,
+                                       w.scale, 1, 4096, 0, 0, ws, nb, stream), 3)
+    res["gqa_long_B2_Hq32_Hkv8_S8192_D128_causal_window4096"] = {
+        "fwd_ms": wfms, "fwd_tflops": wf / wfms / 1e9, "bwd_ms": wbms, "bwd_tflops": 2.5 * wf / wbms / 1e9,
+        "fwd_frac_of_measured_peak": wf / wfms / 1e9 / pk["bf16_tflops"],
+        "bwd_frac_of_measured_peak": 2.5 * wf / wbms / 1e9 / pk["bf16_tflops"]}
     del t, out, lse, dq, dk, dv, ws
 
     # varlen packed batch, D = 64 and 256 (forward; backward for D = 64)

@@ -27,6 +27,8 @@ from .attention import (  # noqa: F401
     varlen_forward,
     varlen_backward,
     kvcache_forward,
+    kvcache_update_forward,
+    logical_cache_rows,
     kv_head_of,
     merge_lse_partials,
 )

@@ -252,6 +252,69 @@ def kvcache_forward(q, k_cache, v_cache, cache_seqlens, scale, causal, rows=None
     return o, lse
 
 
+def logical_cache_rows(cache, b, n, cache_batch_idx=None, block_table=None):
+    """(block, row) address of logical cache rows 0..n-1 of sequence b, and the rows themselves.
+
+    README, ``flash_attn_with_kvcache`` docstring: without a block table the
+    cache is (batch_size_cache, seqlen_cache, nheads_k, headdim) and sequence b
+    reads batch row cache_batch_idx[b] (b itself when no index is given); with a
+    block table the cache is (num_blocks, page_block_size, nheads_k, headdim).
+    Reading where the docstring stops: block_table[b, i] is the physical block
+    that holds logical rows i * page_block_size .. (i + 1) * page_block_size - 1
+    of sequence b, so logical row p sits at (block_table[b, p // page], p % page).
+    """
+    if block_table is not None:
+        page = cache.shape[1]
+        addr = [(int(block_table[b][p // page]), p % page) for p in range(n)]
+    else:
+        bc = b if cache_batch_idx is None else int(cache_batch_idx[b])
+        addr = [(bc, p) for p in range(n)]
+    rows = np.stack([np.asarray(cache[blk, r], dtype=np.float64) for blk, r in addr]) if n > 0 else \
+        np.zeros((0,) + tuple(cache.shape[2:]), dtype=np.float64)
+    return addr, rows
+
+
+def kvcache_update_forward(q, k_cache, v_cache, cache_seqlens, scale, causal, window=(-1, -1), k_new=None,
+                           v_new=None, cache_batch_idx=None, block_table=None):
+    """The full flash_attn_with_kvcache computation (README docstring), without rotary embedding.
+
+    1. If k_new / v_new (B, seqlen_new, nheads_k, headdim) are given, they are
+       written into the caches at logical rows cache_seqlens[b] ..
+       cache_seqlens[b] + seqlen_new - 1 of sequence b ("k is concatenated with
+       k_cache starting at the indices specified by cache_seqlens"; the caches
+       are updated in place, here in copies that are returned).
+    2. Sequence b then attends to its first cache_seqlens[b] + seqlen_new
+       logical rows (addressing: :func:`logical_cache_rows`).
+    3. Attention by the definition, with the bottom-right aligned causal mask
+       and sliding window of :func:`allowed_mask`.
+    Returns O (B, Sq, Hq, headdim), LSE (B, Hq, Sq), k_cache_after, v_cache_after.
+    """
+    B, Sq, Hq, D = q.shape
+    Hkv = k_cache.shape[2]
+    _check_heads(Hq, Hkv)
+    k_after = np.array(k_cache, dtype=np.float64, copy=True)
+    v_after = np.array(v_cache, dtype=np.float64, copy=True)
+    sn = 0 if k_new is None else k_new.shape[1]
+    for b in range(B):
+        start = int(cache_seqlens[b])
+        addr, _ = logical_cache_rows(k_after, b, start + sn, cache_batch_idx, block_table)
+        for s in range(sn):
+            blk, r = addr[start + s]
+            k_after[blk, r] = k_new[b, s]
+            v_after[blk, r] = v_new[b, s]
+    o = np.zeros((B, Sq, Hq, v_cache.shape[3]), dtype=np.float64)
+    lse = np.zeros((B, Hq, Sq), dtype=np.float64)
+    for b in range(B):
+        L = int(cache_seqlens[b]) + sn
+        _, kk = logical_cache_rows(k_after, b, L, cache_batch_idx, block_table)
+        _, vv = logical_cache_rows(v_after, b, L, cache_batch_idx, block_table)
+        mask = allowed_mask(Sq, L, causal, window)
+        for h in range(Hq):
+            hk = kv_head_of(h, Hq, Hkv)
+            o[b, :, h, :], lse[b, h, :], _ = head_forward(q[b, :, h, :], kk[:, hk, :], vv[:, hk, :], scale, mask)
+    return o, lse, k_after, v_after
+
+
 def merge_lse_partials(lse_parts, o_parts):
     """Merge attention results computed over disjoint key sets.
 

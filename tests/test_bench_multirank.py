@@ -64,3 +64,12 @@ def test_reference_arm_runs_on_rank_zero_only():
                         "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""                 # the non-zero rank prints nothing and does no work
+
+
+@pytest.mark.parametrize("Sq,Sk,left,right,causal", [(9, 9, 3, 0, True), (7, 12, 2, 1, False), (12, 7, -1, 2, False),
+                                                     (10, 10, -1, -1, True), (10, 10, -1, -1, False),
+                                                     (8, 8, 2, -1, False), (5, 3, 0, 1, False)])
+def test_window_pair_count_matches_oracle_mask(Sq, Sk, left, right, causal):
+    import bench
+    import oracle
+    assert bench.window_pairs(Sq, Sk, left, right, causal) == oracle.allowed_mask(Sq, Sk, causal, (left, right)).sum()

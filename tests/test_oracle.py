@@ -404,3 +404,98 @@ def test_window_varlen_equals_per_sequence_dense():
         np.testing.assert_array_equal(dq[a:b], gq[0])
         np.testing.assert_array_equal(dk[a:b], gk[0])
         np.testing.assert_array_equal(dv[a:b], gv[0])
+
+
+# ----------------------------------------------------------------------------- KV cache: append, paging, Sq > 1
+
+
+def test_paged_cache_address_matches_hand_derived_rows():
+    want = read_golden("paged_cache_rows_page2.txt")
+    cache = np.zeros((4, 2, 1, 1))
+    for blk in range(4):
+        for r in range(2):
+            cache[blk, r, 0, 0] = 10 * blk + r
+    table = np.array([[2, 0], [3, 1]])
+    for b in range(2):
+        _, rows = oracle.logical_cache_rows(cache, b, 4, block_table=table)
+        assert rows[:, 0, 0].tolist() == want[b]
+
+
+def _cache(B, cap, Hkv, D, lens):
+    kc, vc = np.full((B, cap, Hkv, D), np.nan), np.full((B, cap, Hkv, D), np.nan)
+    for b in range(B):
+        kc[b, :lens[b]] = rnd(lens[b], Hkv, D)
+        vc[b, :lens[b]] = rnd(lens[b], Hkv, D)
+    return kc, vc
+
+
+def test_kvcache_update_equals_dense_on_the_concatenation():
+    # append k_new / v_new at cache_seqlens, then attend causally with several queries: the dense
+    # function on the concatenated keys, bottom-right aligned
+    B, cap, Hq, Hkv, D, Sq, Sn = 3, 24, 4, 2, 8, 5, 3
+    lens = np.array([0, 9, 21])
+    kc, vc = _cache(B, cap, Hkv, D, lens)
+    q, kn, vn = rnd(B, Sq, Hq, D), rnd(B, Sn, Hkv, D), rnd(B, Sn, Hkv, D)
+    for causal, window in ((True, (-1, -1)), (False, (-1, -1)), (True, (4, -1)), (False, (2, 1))):
+        o, lse, ka, va = oracle.kvcache_update_forward(q, kc, vc, lens, 0.4, causal, window, kn, vn)
+        for b in range(B):
+            L = lens[b]
+            kk = np.concatenate([kc[b, :L], kn[b]])[None]
+            vv = np.concatenate([vc[b, :L], vn[b]])[None]
+            od, ld = oracle.mha_forward(q[b:b + 1], kk, vv, 0.4, causal, window)
+            np.testing.assert_allclose(o[b], od[0], rtol=0, atol=1e-14)
+            np.testing.assert_array_equal(np.isneginf(lse[b]), np.isneginf(ld[0]))
+            np.testing.assert_allclose(lse[b][np.isfinite(ld[0])], ld[0][np.isfinite(ld[0])], rtol=0, atol=1e-14)
+            # the caches were updated in place at rows L .. L + Sn - 1 and nowhere else
+            np.testing.assert_array_equal(ka[b, L:L + Sn], kn[b])
+            np.testing.assert_array_equal(va[b, L:L + Sn], vn[b])
+            np.testing.assert_array_equal(np.isnan(ka[b, L + Sn:]), np.isnan(kc[b, L + Sn:]))
+
+
+def test_kvcache_update_paged_equals_contiguous():
+    # scatter a contiguous cache into pages through a random block table: same result, and the append
+    # lands in the right physical rows
+    B, cap, Hq, Hkv, D, page = 3, 16, 2, 1, 8, 4
+    lens = np.array([5, 12, 0])
+    kc, vc = _cache(B, cap, Hkv, D, lens)
+    nblk = B * cap // page
+    perm = np.random.default_rng(5).permutation(nblk)
+    table = perm.reshape(B, cap // page)
+    kp, vp = np.zeros((nblk, page, Hkv, D)), np.zeros((nblk, page, Hkv, D))
+    for b in range(B):
+        for i in range(cap // page):
+            kp[table[b, i]] = kc[b, i * page:(i + 1) * page]
+            vp[table[b, i]] = vc[b, i * page:(i + 1) * page]
+    q, kn, vn = rnd(B, 3, Hq, D), rnd(B, 2, Hkv, D), rnd(B, 2, Hkv, D)
+    o1, l1, ka1, _ = oracle.kvcache_update_forward(q, kc, vc, lens, 0.3, True, (-1, -1), kn, vn)
+    o2, l2, ka2, _ = oracle.kvcache_update_forward(q, kp, vp, lens, 0.3, True, (-1, -1), kn, vn, block_table=table)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    for b in range(B):
+        for i in range(cap // page):
+            np.testing.assert_array_equal(ka2[table[b, i]], ka1[b, i * page:(i + 1) * page])
+
+
+def test_kvcache_update_with_batch_index_reads_the_indexed_rows():
+    B, cap, Hq, Hkv, D = 3, 10, 2, 2, 8
+    kc, vc = _cache(4, cap, Hkv, D, [10, 10, 10, 10])
+    idx = np.array([3, 0, 2])
+    lens = np.array([4, 10, 7])
+    q = rnd(B, 2, Hq, D)
+    o, lse, _, _ = oracle.kvcache_update_forward(q, kc, vc, lens, 0.5, True, cache_batch_idx=idx)
+    o_ref, l_ref = oracle.kvcache_forward(q, kc[idx], vc[idx], lens, 0.5, True)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(lse, l_ref)
+
+
+def test_kvcache_update_without_new_keys_is_kvcache_forward():
+    B, cap, Hq, Hkv, D = 2, 12, 4, 1, 8
+    lens = np.array([12, 3])
+    kc, vc = _cache(B, cap, Hkv, D, lens)
+    q = rnd(B, 4, Hq, D)
+    for causal in (False, True):
+        o, lse, ka, _ = oracle.kvcache_update_forward(q, kc, vc, lens, 0.5, causal)
+        o_ref, l_ref = oracle.kvcache_forward(q, kc, vc, lens, 0.5, causal)
+        np.testing.assert_array_equal(o, o_ref)
+        np.testing.assert_array_equal(lse, l_ref)
+        np.testing.assert_array_equal(np.isnan(ka), np.isnan(kc))

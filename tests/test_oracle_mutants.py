@@ -135,3 +135,36 @@ def test_window_mask_mutants_are_caught(monkeypatch, mutant):
             caught += 1
     assert caught > 0
     _fails(pins.test_window_forward_matches_sliced_sdpa, 9, 14, (2, 1))
+
+
+_ORIG_ROWS = A.logical_cache_rows
+
+
+def _paged_rows_swapped(cache, b, n, cache_batch_idx=None, block_table=None):
+    # page index and offset exchanged
+    if block_table is None:
+        return _ORIG_ROWS(cache, b, n, cache_batch_idx, block_table)
+    page = cache.shape[1]
+    addr = [(int(block_table[b][p % page]), p // page) for p in range(n)]
+    rows = np.stack([np.asarray(cache[k, r], dtype=np.float64) for k, r in addr])
+    return addr, rows
+
+
+def _append_one_row_late(cache, b, n, cache_batch_idx=None, block_table=None):
+    # every logical row addressed one row further on (kept inside the capacity)
+    addr, _ = _ORIG_ROWS(cache, b, n, cache_batch_idx, block_table)
+    addr = [(k, min(r + 1, cache.shape[1] - 1)) for k, r in addr]
+    rows = np.stack([np.asarray(cache[k, r], dtype=np.float64) for k, r in addr]) if n > 0 else \
+        np.zeros((0,) + tuple(cache.shape[2:]))
+    return addr, rows
+
+
+def test_paged_address_mutant_is_caught(monkeypatch):
+    monkeypatch.setattr(A, "logical_cache_rows", _paged_rows_swapped)
+    monkeypatch.setattr(oracle, "logical_cache_rows", _paged_rows_swapped)
+    _fails(pins.test_paged_cache_address_matches_hand_derived_rows)
+
+
+def test_append_offset_mutant_is_caught(monkeypatch):
+    monkeypatch.setattr(A, "logical_cache_rows", _append_one_row_late)
+    _fails(pins.test_kvcache_update_equals_dense_on_the_concatenation)
