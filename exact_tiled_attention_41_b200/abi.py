@@ -32,6 +32,7 @@ EXPORTS = (
     "fa_profile_begin", "fa_profile_read",
     "fa_fwd_kvcache_noalloc", "fa_fwd_kvcache_noalloc_scratch_bytes", "fa_debug_exp2_selftest",
     "fa_fwd_ex", "fa_bwd_ex", "fa_varlen_fwd_ex", "fa_varlen_bwd_ex",
+    "fa_fwd_kvcache_ex", "fa_fwd_kvcache_ex_workspace_size",
 )
 
 FA_KERNEL_FWD = 0
@@ -69,6 +70,9 @@ _SIGS = {
     "fa_bwd_ex": (_I, [_P] * 9 + [_I] * 6 + [_F, _I, _I, _I, _I, _P, _Z, _P]),
     "fa_varlen_fwd_ex": (_I, [_P] * 7 + [_I] * 8 + [_F, _I, _I, _I, _P, _Z, _P]),
     "fa_varlen_bwd_ex": (_I, [_P] * 11 + [_I] * 8 + [_F, _I, _I, _I, _I, _P, _Z, _P]),
+    "fa_fwd_kvcache_ex_workspace_size": (_Z, [_I] * 8),
+    "fa_fwd_kvcache_ex": (_I, [_P] * 6 + [_I] + [_P] * 2 + [_I] * 3 + [_P] * 2 + [_I] * 5 + [_F] + [_I] * 4
+                          + [_P, _Z, _P]),
 }
 
 _lib = None
@@ -205,6 +209,21 @@ def fa_varlen_bwd_ex(q, k, v, out, dout, lse, dq, dk, dv, cu_seqlens_q, cu_seqle
                                    max_seqlen_k, total_q, total_k, Hq, Hkv, D, float(softmax_scale),
                                    int(bool(causal)), int(window_left), int(window_right), int(bool(deterministic)),
                                    _ptr(workspace), workspace_bytes, _stream(stream))
+
+
+def fa_fwd_kvcache_ex_workspace_size(B, Hq, Hkv, Sq, D, cache_capacity, max_blocks_per_seq, num_splits) -> int:
+    return load().fa_fwd_kvcache_ex_workspace_size(B, Hq, Hkv, Sq, D, cache_capacity, max_blocks_per_seq, num_splits)
+
+
+def fa_fwd_kvcache_ex(q, k_cache, v_cache, cache_seqlens, k_new, v_new, seqlen_new, cache_batch_idx, block_table,
+                      max_blocks_per_seq, cache_batch, cache_capacity, out, lse, B, Hq, Hkv, Sq, D, softmax_scale,
+                      causal, window_left, window_right, num_splits, workspace, workspace_bytes, stream=None) -> int:
+    return load().fa_fwd_kvcache_ex(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens), _ptr(k_new),
+                                    _ptr(v_new), int(seqlen_new), _ptr(cache_batch_idx), _ptr(block_table),
+                                    int(max_blocks_per_seq), int(cache_batch), int(cache_capacity), _ptr(out),
+                                    _ptr(lse), B, Hq, Hkv, Sq, D, float(softmax_scale), int(bool(causal)),
+                                    int(window_left), int(window_right), int(num_splits), _ptr(workspace),
+                                    workspace_bytes, _stream(stream))
 
 
 def fa_get_device_status(stream=None) -> int:

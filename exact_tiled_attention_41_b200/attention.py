@@ -116,20 +116,44 @@ def flash_attn_varlen_backward(dout, q, k, v, out, lse, cu_seqlens_q, cu_seqlens
 
 
 def flash_attn_with_kvcache(q, k_cache, v_cache, cache_seqlens, softmax_scale=None, causal=False, num_splits=0,
-                            return_lse=True):
-    """Decode against a contiguous cache: returns (out (B, Sq, Hq, D), lse (B, Hq, Sq) or None)."""
+                            return_lse=True, k=None, v=None, cache_batch_idx=None, block_table=None,
+                            window_size=(-1, -1)):
+    """Attention of new queries against a KV cache (README, flash_attn_with_kvcache docstring).
+
+    q (B, Sq, Hq, D); caches (B_cache, capacity, Hkv, D), or pages (num_blocks, page_block_size, Hkv, D)
+    with block_table (B, max_blocks_per_seq) int32; cache_seqlens int32 (B,) or an int.  If k / v
+    (B, seqlen_new, Hkv, D) are given they are written into the caches in place at cache_seqlens first.
+    Returns (out (B, Sq, Hq, D), lse (B, Hq, Sq) or None).
+    """
     for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
         _check(t, n)
-    _check(cache_seqlens, "cache_seqlens", torch.int32)
     B, Sq, Hq, D = q.shape
-    cap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    if isinstance(cache_seqlens, int):
+        cache_seqlens = torch.full((B,), cache_seqlens, dtype=torch.int32, device=q.device)
+    _check(cache_seqlens, "cache_seqlens", torch.int32)
+    if (k is None) != (v is None):
+        raise ValueError("k and v must be given together")
+    sn = 0
+    if k is not None:
+        _check(k, "k")
+        _check(v, "v")
+        sn = k.shape[1]
+    if cache_batch_idx is not None:
+        _check(cache_batch_idx, "cache_batch_idx", torch.int32)
+    max_blocks = 0
+    if block_table is not None:
+        _check(block_table, "block_table", torch.int32)
+        max_blocks = block_table.shape[1]
+    cache_batch, cap, Hkv = k_cache.shape[0], k_cache.shape[1], k_cache.shape[2]
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
     out = torch.empty_like(q)
     lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device) if return_lse else None
-    nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, Sq, cap, D, num_splits)
+    nb = abi.fa_fwd_kvcache_ex_workspace_size(B, Hq, Hkv, Sq, D, cap, max_blocks, num_splits)
     ws = _workspace(nb, q.device)
-    _raise(abi.fa_fwd_kvcache(q, k_cache, v_cache, cache_seqlens, out, lse, B, Hq, Hkv, Sq, cap, D, scale, causal,
-                              num_splits, ws, nb), "fa_fwd_kvcache")
+    left, right = _window(window_size)
+    _raise(abi.fa_fwd_kvcache_ex(q, k_cache, v_cache, cache_seqlens, k, v, sn, cache_batch_idx, block_table,
+                                 max_blocks, cache_batch, cap, out, lse, B, Hq, Hkv, Sq, D, scale, causal, left, right,
+                                 num_splits, ws, nb), "fa_fwd_kvcache_ex")
     return out, lse
 
 

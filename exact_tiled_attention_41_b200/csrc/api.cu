@@ -347,57 +347,90 @@ int fa_varlen_bwd_ex(const void* q, const void* k, const void* v, const void* ou
 }
 
 // ----------------------------------------------------------------------- KV-cache decode
-static int validate_kvcache(int B, int Hq, int Hkv, int Sq, int cap, int D, float scale, int num_splits) {
-    if (B <= 0 || cap <= 0 || num_splits < 0) return FA_ERR_INVALID_ARG;
-    if (Sq != 1) return FA_ERR_INVALID_ARG;
-    int st = check_heads(Hq, Hkv, D, scale);
+// A contiguous cache of B rows; `paged_tag` stands in for the block table when only shapes are checked.
+static KvCall plain_kv_call(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_seqlens,
+                            void* out, float* lse, int B, int Hq, int Hkv, int Sq, int cache_capacity, int D,
+                            float softmax_scale, int causal, int num_splits) {
+    KvCall c = {};
+    c.q = q;
+    c.k_cache = const_cast<void*>(k_cache);
+    c.v_cache = const_cast<void*>(v_cache);
+    c.cache_seqlens = cache_seqlens;
+    c.cache_batch = B;
+    c.cache_capacity = cache_capacity;
+    c.out = out;
+    c.lse = lse;
+    c.B = B;
+    c.Hq = Hq;
+    c.Hkv = Hkv;
+    c.Sq = Sq;
+    c.D = D;
+    c.scale = softmax_scale;
+    c.causal = causal;
+    c.window_left = -1;
+    c.window_right = -1;
+    c.num_splits = num_splits;
+    return c;
+}
+
+static int run_kv_call(const KvCall& c, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    int st = kvcache_validate(c, true);
     if (st != FA_OK) return st;
-    if (D != 128 && D != 64) return FA_ERR_UNSUPPORTED;
-    if (Hq / Hkv > 8) return FA_ERR_UNSUPPORTED;
-    if ((st = check_tokens(static_cast<long long>(B) * cap, Hkv, D)) != FA_OK) return st;
-    return FA_OK;
+    if (!workspace) return FA_ERR_INVALID_ARG;
+    if (!aligned256(workspace)) return FA_ERR_ALIGNMENT;
+    const int chunk = kvcache_chunk(c, 148);
+    if (workspace_bytes < kvcache_workspace_bytes(c, chunk)) return FA_ERR_WORKSPACE;
+    Device dev;
+    if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
+    return kvcache_launch(c, chunk, workspace, dev, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Sq, int cache_capacity, int D, int num_splits) {
-    if (validate_kvcache(B, Hq, Hkv, Sq, cache_capacity, D, 1.0f, num_splits) != FA_OK) return 0;
-    const int chunk = decode_chunk_size(B, Hkv, cache_capacity, num_splits, 148);
-    return decode_workspace_bytes(B, Hq, Hkv, cache_capacity, D, chunk);
+    KvCall c = plain_kv_call(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, Sq, cache_capacity, D,
+                             1.0f, 0, num_splits);
+    if (kvcache_validate(c, false) != FA_OK) return 0;
+    return kvcache_workspace_bytes(c, kvcache_chunk(c, 148));
 }
 
 int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_seqlens, void* out,
                    float* lse, int B, int Hq, int Hkv, int Sq, int cache_capacity, int D, float softmax_scale,
                    int causal, int num_splits, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-    (void)causal;  // one query row sees every valid key under the bottom-right causal rule
-    int st = validate_kvcache(B, Hq, Hkv, Sq, cache_capacity, D, softmax_scale, num_splits);
-    if (st != FA_OK) return st;
-    if (!q || !k_cache || !v_cache || !cache_seqlens || !out || !workspace) return FA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out)) return FA_ERR_ALIGNMENT;
-    if (lse && !aligned16(lse)) return FA_ERR_ALIGNMENT;
-    if (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) return FA_ERR_ALIGNMENT;
-    if (!aligned256(workspace)) return FA_ERR_ALIGNMENT;
-    const int chunk = decode_chunk_size(B, Hkv, cache_capacity, num_splits, 148);
-    if (workspace_bytes < decode_workspace_bytes(B, Hq, Hkv, cache_capacity, D, chunk)) return FA_ERR_WORKSPACE;
-    Device dev;
-    if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
-    Decode d;
-    d.q = q;
-    d.k_cache = k_cache;
-    d.v_cache = v_cache;
-    d.seqlens = cache_seqlens;
-    d.out = out;
-    d.lse = lse;
-    d.B = B;
-    d.Hq = Hq;
-    d.Hkv = Hkv;
-    d.cap = cache_capacity;
-    d.D = D;
-    d.scale = softmax_scale;
-    d.chunk = chunk;
-    d.max_chunks = (cache_capacity + chunk - 1) / chunk;
-    const size_t rows = static_cast<size_t>(B) * Hkv * d.max_chunks * (Hq / Hkv);
-    d.part_o = static_cast<float*>(workspace);
-    d.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + ((rows * D * 4 + 255) & ~size_t(255)));
-    return launch_decode(d, dev, static_cast<cudaStream_t>(stream));
+    const KvCall c = plain_kv_call(q, k_cache, v_cache, cache_seqlens, out, lse, B, Hq, Hkv, Sq, cache_capacity, D,
+                                   softmax_scale, causal, num_splits);
+    return run_kv_call(c, workspace, workspace_bytes, stream);
+}
+
+size_t fa_fwd_kvcache_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int D, int cache_capacity,
+                                        int max_blocks_per_seq, int num_splits) {
+    KvCall c = plain_kv_call(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, Sq, cache_capacity, D,
+                             1.0f, 0, num_splits);
+    if (max_blocks_per_seq < 0) return 0;
+    static const int32_t paged_tag = 0;
+    if (max_blocks_per_seq > 0) {
+        c.block_table = &paged_tag;   // only its presence matters for the sizes
+        c.max_blocks_per_seq = max_blocks_per_seq;
+    }
+    if (kvcache_validate(c, false) != FA_OK) return 0;
+    return kvcache_workspace_bytes(c, kvcache_chunk(c, 148));
+}
+
+int fa_fwd_kvcache_ex(const void* q, void* k_cache, void* v_cache, const int32_t* cache_seqlens, const void* k_new,
+                      const void* v_new, int seqlen_new, const int32_t* cache_batch_idx, const int32_t* block_table,
+                      int max_blocks_per_seq, int cache_batch, int cache_capacity, void* out, float* lse, int B,
+                      int Hq, int Hkv, int Sq, int D, float softmax_scale, int causal, int window_left,
+                      int window_right, int num_splits, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+    KvCall c = plain_kv_call(q, k_cache, v_cache, cache_seqlens, out, lse, B, Hq, Hkv, Sq, cache_capacity, D,
+                             softmax_scale, causal, num_splits);
+    c.k_new = k_new;
+    c.v_new = v_new;
+    c.seqlen_new = seqlen_new;
+    c.cache_batch_idx = cache_batch_idx;
+    c.block_table = block_table;
+    c.max_blocks_per_seq = max_blocks_per_seq;
+    c.cache_batch = cache_batch;
+    c.window_left = window_left;
+    c.window_right = window_right;
+    return run_kv_call(c, workspace, workspace_bytes, stream);
 }
 
 // ----------------------------------------------------------------------- diagnostics

@@ -58,24 +58,31 @@ int launch_bwd_dq(const Problem& pr, const void* dout, const float* lse2, const 
 int launch_bwd(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
                void* dv, void* workspace, bool deterministic, const Device& dev, cudaStream_t stream);
 
-struct Decode {
-    const void* q;            // [B, 1, Hq, D]
-    const void* k_cache;      // [B, cap, Hkv, D]
-    const void* v_cache;
-    const int32_t* seqlens;   // device [B]
-    void* out;                // [B, 1, Hq, D]
-    float* lse;               // [B, Hq, 1] or NULL
-    int B, Hq, Hkv, cap, D;
+// One flash_attn_with_kvcache call as the C ABI receives it (README, flash_attn_with_kvcache docstring).
+struct KvCall {
+    const void* q;                   // [B, Sq, Hq, D]
+    void* k_cache;                   // contiguous [cache_batch, cache_capacity, Hkv, D];
+    void* v_cache;                   // paged [cache_batch = num_blocks, cache_capacity = page_block_size, Hkv, D]
+    const int32_t* cache_seqlens;    // device [B]: keys already in the cache
+    const void* k_new;               // [B, seqlen_new, Hkv, D] appended at cache_seqlens, or NULL
+    const void* v_new;
+    int seqlen_new;
+    const int32_t* cache_batch_idx;  // device [B] or NULL (contiguous caches only)
+    const int32_t* block_table;      // device [B, max_blocks_per_seq] or NULL
+    int max_blocks_per_seq;
+    int cache_batch, cache_capacity;
+    void* out;                       // [B, Sq, Hq, D]
+    float* lse;                      // [B, Hq, Sq] or NULL
+    int B, Hq, Hkv, Sq, D;
     float scale;
-    int chunk;                // keys per split (multiple of 64)
-    int max_chunks;           // ceil(cap / chunk)
-    float* part_o;            // [B, Hkv, max_chunks, group, D]
-    float* part_lse;          // [B, Hkv, max_chunks, group]
+    int causal, window_left, window_right, num_splits;
 };
 
-int decode_chunk_size(int B, int Hkv, int cap, int num_splits, int num_sms);
-size_t decode_workspace_bytes(int B, int Hq, int Hkv, int cap, int D, int chunk);
-int launch_decode(const Decode& d, const Device& dev, cudaStream_t stream);
+int kvcache_validate(const KvCall& c, bool pointers);         // FA status, no CUDA calls
+int kvcache_chunk(const KvCall& c, int num_sms);              // keys per split (multiple of 64)
+int kvcache_chunk_limit(const KvCall& c);                     // keys one sequence can hold
+size_t kvcache_workspace_bytes(const KvCall& c, int chunk);   // float32 partial outputs and LSEs
+int kvcache_launch(const KvCall& c, int chunk, void* workspace, const Device& dev, cudaStream_t stream);
 
 int launch_wait_selftest(unsigned long long timeout_ns, const Device& dev, cudaStream_t stream);
 int launch_exp2_selftest(const float* x, float* y, int n, cudaStream_t stream);

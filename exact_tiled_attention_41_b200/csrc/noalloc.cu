@@ -49,21 +49,34 @@ extern "C" int fa_fwd_kvcache_noalloc(const void* q, const void* k_cache, const 
                                       const int32_t* cache_seqlens, void* out, float* lse, int B, int Hq, int Hkv,
                                       int Sq, int cache_capacity, int D, float softmax_scale, int causal,
                                       int num_splits, fa_stream_t stream) {
-    (void)causal;  // one query row sees every valid key under the bottom-right causal rule
-    if (!q || !k_cache || !v_cache || !cache_seqlens || !out) return FA_ERR_INVALID_ARG;
-    if (B <= 0 || cache_capacity <= 0 || num_splits < 0 || Sq != 1) return FA_ERR_INVALID_ARG;
-    if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || !(softmax_scale > 0.f)) return FA_ERR_INVALID_ARG;
-    if ((D != 64 && D != 128) || Hq / Hkv > 8) return FA_ERR_UNSUPPORTED;
-    if (static_cast<long long>(B) * cache_capacity > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
-    auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    if (!a16(q) || !a16(k_cache) || !a16(v_cache) || !a16(out) || (lse && !a16(lse))) return FA_ERR_ALIGNMENT;
-    if (reinterpret_cast<uintptr_t>(cache_seqlens) & 3u) return FA_ERR_ALIGNMENT;
+    KvCall c = {};
+    c.q = q;
+    c.k_cache = const_cast<void*>(k_cache);
+    c.v_cache = const_cast<void*>(v_cache);
+    c.cache_seqlens = cache_seqlens;
+    c.cache_batch = B;
+    c.cache_capacity = cache_capacity;
+    c.out = out;
+    c.lse = lse;
+    c.B = B;
+    c.Hq = Hq;
+    c.Hkv = Hkv;
+    c.Sq = Sq;
+    c.D = D;
+    c.scale = softmax_scale;
+    c.causal = causal;
+    c.window_left = -1;
+    c.window_right = -1;
+    c.num_splits = num_splits;
+    const int st0 = kvcache_validate(c, true);
+    if (st0 != FA_OK) return st0;
 
     // Split size: the usual choice, made coarser (auto mode only) until the partials fit the fixed array.
-    int chunk = decode_chunk_size(B, Hkv, cache_capacity, num_splits, 148);
-    while (decode_workspace_bytes(B, Hq, Hkv, cache_capacity, D, chunk) > kNoAllocScratchBytes) {
-        if (num_splits > 0 || chunk >= cache_capacity) return FA_ERR_WORKSPACE;   // beyond the fixed maximum
-        chunk = chunk * 2 > cache_capacity ? (cache_capacity + 63) / 64 * 64 : chunk * 2;
+    const int cap = kvcache_chunk_limit(c);
+    int chunk = kvcache_chunk(c, 148);
+    while (kvcache_workspace_bytes(c, chunk) > kNoAllocScratchBytes) {
+        if (num_splits > 0 || chunk >= cap) return FA_ERR_WORKSPACE;   // beyond the fixed maximum
+        chunk = chunk * 2 > cap ? (cap + 63) / 64 * 64 : chunk * 2;
     }
 
     Device dev;
@@ -71,24 +84,5 @@ extern "C" int fa_fwd_kvcache_noalloc(const void* q, const void* k_cache, const 
     void* scratch = nullptr;
     const int st = scratch_for_current_device(dev, &scratch);
     if (st != FA_OK) return st;
-
-    Decode d;
-    d.q = q;
-    d.k_cache = k_cache;
-    d.v_cache = v_cache;
-    d.seqlens = cache_seqlens;
-    d.out = out;
-    d.lse = lse;
-    d.B = B;
-    d.Hq = Hq;
-    d.Hkv = Hkv;
-    d.cap = cache_capacity;
-    d.D = D;
-    d.scale = softmax_scale;
-    d.chunk = chunk;
-    d.max_chunks = (cache_capacity + chunk - 1) / chunk;
-    const size_t rows = static_cast<size_t>(B) * Hkv * d.max_chunks * (Hq / Hkv);
-    d.part_o = static_cast<float*>(scratch);
-    d.part_lse = reinterpret_cast<float*>(static_cast<char*>(scratch) + ((rows * D * 4 + 255) & ~size_t(255)));
-    return launch_decode(d, dev, static_cast<cudaStream_t>(stream));
+    return kvcache_launch(c, chunk, scratch, dev, static_cast<cudaStream_t>(stream));
 }

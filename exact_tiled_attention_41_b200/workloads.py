@@ -110,6 +110,58 @@ def kvcache(B, Hq, Hkv, D, capacity, lo, hi, seed=0, Sq=1, nan_guard=True, name=
     return Workload(name or f"kvcache_B{B}_Hq{Hq}_Hkv{Hkv}_D{D}", "kvcache", False, 1.0 / math.sqrt(D), t, meta)
 
 
+def kvcache_update(B, Sq, Hq, Hkv, D, capacity, lengths, seqlen_new=0, page=0, seed=0, cache_batch_idx=None,
+                   cache_batch=None, spare_blocks=3, name=None) -> Workload:
+    """A cache for one flash_attn_with_kvcache call: Sq new queries, optional k / v to append.
+
+    Contiguous (page = 0): caches (cache_batch or B, capacity, Hkv, D); sequence b lives in cache row
+    cache_batch_idx[b] (b without an index).  Paged (page > 0, capacity a multiple of page): caches
+    (num_blocks, page, Hkv, D) with num_blocks = B * capacity / page + spare_blocks, and a block table
+    (B, capacity / page) drawn as a random permutation of the blocks.  Logical rows below
+    lengths[b] hold N(0, 1) values, every other row NaN (nothing may read them).  Draw order: block
+    permutation, q, K rows, V rows, k_new, v_new.
+    """
+    g = torch.Generator("cpu").manual_seed(seed)
+    lens = torch.as_tensor(lengths, dtype=torch.int64)
+    t = {}
+    if page > 0:
+        assert capacity % page == 0
+        nblk_seq = capacity // page
+        nblk = B * nblk_seq + spare_blocks
+        perm = torch.randperm(nblk, generator=g)[:B * nblk_seq]
+        table = perm.reshape(B, nblk_seq).to(torch.int32)
+        kc = torch.full((nblk, page, Hkv, D), BF16_NAN, dtype=torch.bfloat16)
+        vc = torch.full((nblk, page, Hkv, D), BF16_NAN, dtype=torch.bfloat16)
+        t["block_table"] = table
+
+        def rows(cache, b, L, vals):
+            for p0 in range(0, L, page):
+                n = min(page, L - p0)
+                cache[int(table[b, p0 // page]), :n] = vals[p0:p0 + n]
+    else:
+        nb = cache_batch if cache_batch is not None else B
+        kc = torch.full((nb, capacity, Hkv, D), BF16_NAN, dtype=torch.bfloat16)
+        vc = torch.full((nb, capacity, Hkv, D), BF16_NAN, dtype=torch.bfloat16)
+        idx = torch.arange(B) if cache_batch_idx is None else torch.as_tensor(cache_batch_idx, dtype=torch.int64)
+        if cache_batch_idx is not None:
+            t["cache_batch_idx"] = idx.to(torch.int32)
+
+        def rows(cache, b, L, vals):
+            cache[int(idx[b]), :L] = vals
+    q = _randn(g, (B, Sq, Hq, D))
+    for b in range(B):
+        rows(kc, b, int(lens[b]), _randn(g, (int(lens[b]), Hkv, D)))
+    for b in range(B):
+        rows(vc, b, int(lens[b]), _randn(g, (int(lens[b]), Hkv, D)))
+    if seqlen_new > 0:
+        t["k_new"] = _randn(g, (B, seqlen_new, Hkv, D))
+        t["v_new"] = _randn(g, (B, seqlen_new, Hkv, D))
+    t.update(q=q, k_cache=kc, v_cache=vc, cache_seqlens=lens.to(torch.int32))
+    meta = dict(B=B, Sq=Sq, Hq=Hq, Hkv=Hkv, D=D, capacity=capacity, page=page, seqlen_new=seqlen_new)
+    return Workload(name or f"kvcache_update_B{B}_Sq{Sq}_Hq{Hq}_Hkv{Hkv}_D{D}", "kvcache", False,
+                    1.0 / math.sqrt(D), t, meta)
+
+
 # The five workloads: sizes as stated for each configuration.
 def tiny(causal: bool, seed=0) -> Workload:
     """B=1, Hq=Hkv=2, Sq=Sk=128, D=64."""

@@ -63,7 +63,7 @@ typedef void* fa_stream_t; /* a cudaStream_t */
 
 enum fa_status {
     FA_OK = 0,
-    FA_ERR_INVALID_ARG = 1,  /* non-positive sizes, Hq % Hkv != 0, NULL pointer, bad Sq for kvcache */
+    FA_ERR_INVALID_ARG = 1,  /* non-positive sizes, Hq % Hkv != 0, NULL pointer, bad page size / table */
     FA_ERR_UNSUPPORTED = 2,  /* head dim outside {64, 128, 256}, or a size beyond the int32 index range */
     FA_ERR_ALIGNMENT = 3,    /* a tensor pointer is not 16-byte aligned / workspace not 256-byte aligned */
     FA_ERR_WORKSPACE = 4,    /* workspace_bytes smaller than the *_workspace_size() figure */
@@ -184,12 +184,13 @@ FA_API int fa_varlen_bwd_ex(const void* q, const void* k, const void* v, const v
  *   cache_seqlens DEVICE int32 [B]: batch row b uses keys 0 .. cache_seqlens[b]-1,
  *   each in [0, cache_capacity]; rows beyond it are never read into the result.
  *   out [B, Sq, Hq, D]   lse [B, Hq, Sq] float32, or NULL if not wanted.
- * Sq must be 1 in this version (causal is then irrelevant: the single query
- * sees every valid key).  num_splits = 0 picks the split of the cache
+ * Sq >= 1 new query tokens per row; with causal != 0 token i of row b sees
+ * keys 0 .. i + cache_seqlens[b] - Sq (bottom-right aligned; for Sq = 1 that is
+ * every valid key).  num_splits = 0 picks the split of the cache
  * automatically; > 0 asks for that many splits of cache_capacity.  The result
  * does not depend on the split except through float32 rounding.
  * Workspace (fa_fwd_kvcache_workspace_size): float32 partial outputs and LSEs.
- * No backward (the docstring states the same).
+ * Head dims 64 and 128.  No backward (the docstring states the same).
  */
 FA_API size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Sq, int cache_capacity, int D, int num_splits);
 FA_API int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_seqlens,
@@ -197,6 +198,45 @@ FA_API int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cach
                    int B, int Hq, int Hkv, int Sq, int cache_capacity, int D,
                    float softmax_scale, int causal, int num_splits,
                    void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/* ------------------------------------------------------------------------- KV-cache: append, pages, windows
+ * fa_fwd_kvcache_ex: the rest of flash_attn_with_kvcache (README docstring),
+ * without rotary embedding.  In order, on `stream`:
+ *  1. If k_new / v_new [B, seqlen_new, Hkv, D] are given (both, seqlen_new > 0),
+ *     they are written into k_cache / v_cache IN PLACE at logical rows
+ *     cache_seqlens[b] .. cache_seqlens[b] + seqlen_new - 1 of sequence b.
+ *     Rows past what the sequence can hold are not written.  cache_seqlens is
+ *     not modified (the caller advances it).
+ *  2. Sequence b attends to its first min(cache_seqlens[b] + seqlen_new, cap)
+ *     logical rows, with the bottom-right aligned causal mask and sliding window
+ *     of fa_fwd_ex, where cap = cache_capacity (contiguous) or
+ *     max_blocks_per_seq * page_block_size (paged).
+ * Cache layouts:
+ *  - contiguous (block_table = NULL): caches [cache_batch, cache_capacity, Hkv, D];
+ *    sequence b uses cache row cache_batch_idx[b] (DEVICE int32 [B]) or b when
+ *    cache_batch_idx is NULL.  With repeated indices and k_new given, which
+ *    sequence's rows end up in the cache is unspecified (as in the docstring).
+ *  - paged: caches [cache_batch = num_blocks, cache_capacity = page_block_size,
+ *    Hkv, D], page_block_size a multiple of 256 (README); block_table DEVICE
+ *    int32 [B, max_blocks_per_seq]: logical rows i*page .. i*page+page-1 of
+ *    sequence b live in block block_table[b][i] (the reading taken of the
+ *    docstring's block_table).  cache_batch_idx must then be NULL.
+ *  q [B, Sq, Hq, D] and out [B, Sq, Hq, D]; lse [B, Hq, Sq] float32 or NULL.
+ * A block id or cache_batch_idx entry outside the cache is not dereferenced:
+ * the kernels record FA_ERR_INVALID_ARG in the device status word
+ * (fa_get_device_status) and such rows read as zeros / the sequence as empty.
+ * Workspace: fa_fwd_kvcache_ex_workspace_size(B, Hq, Hkv, Sq, D, cache_capacity,
+ * max_blocks_per_seq (0 for a contiguous cache), num_splits).
+ */
+FA_API size_t fa_fwd_kvcache_ex_workspace_size(int B, int Hq, int Hkv, int Sq, int D, int cache_capacity,
+                                               int max_blocks_per_seq, int num_splits);
+FA_API int fa_fwd_kvcache_ex(const void* q, void* k_cache, void* v_cache, const int32_t* cache_seqlens,
+                             const void* k_new, const void* v_new, int seqlen_new,
+                             const int32_t* cache_batch_idx, const int32_t* block_table, int max_blocks_per_seq,
+                             int cache_batch, int cache_capacity,
+                             void* out, float* lse, int B, int Hq, int Hkv, int Sq, int D,
+                             float softmax_scale, int causal, int window_left, int window_right, int num_splits,
+                             void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /* ------------------------------------------------------------------------- KV-cache decode without caller memory
  * fa_fwd_kvcache_noalloc: the same computation as fa_fwd_kvcache, for callers
@@ -217,7 +257,7 @@ FA_API int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cach
  *     Nothing in it needs to start at zero; each call writes what it reads.
  *   - With num_splits = 0 the split is chosen as for fa_fwd_kvcache and made
  *     coarser until the partials fit.  If they cannot fit (an explicit
- *     num_splits too large, or B * Hq * (D + 1) * 4 bytes beyond the array),
+ *     num_splits too large, or B * Sq * Hq * (D + 1) * 4 bytes beyond the array),
  *     the call returns FA_ERR_WORKSPACE and launches nothing.
  */
 FA_API size_t fa_fwd_kvcache_noalloc_scratch_bytes(void);

@@ -123,7 +123,7 @@ def test_kvcache_argument_rules(lib):
     assert need > 0
     args = [FAKE, FAKE, FAKE, FAKE, FAKE, None, 64, 32, 8, 1, 16384, 128, 0.1, 0, 0, FAKE, need, S0]
     bad_sq = list(args)
-    bad_sq[9] = 2                                 # one query per row in this version
+    bad_sq[9] = 0                                 # at least one query token per row
     assert abi.fa_fwd_kvcache(*bad_sq) == abi.FA_ERR_INVALID_ARG
     small = list(args)
     small[16] = need - 1
@@ -134,6 +134,41 @@ def test_kvcache_argument_rules(lib):
     # more splits need more partial storage
     assert abi.fa_fwd_kvcache_workspace_size(64, 32, 8, 1, 16384, 128, 64) > abi.fa_fwd_kvcache_workspace_size(
         64, 32, 8, 1, 16384, 128, 4)
+
+
+def _kv_ex(**kw):
+    a = dict(q=FAKE, k_cache=FAKE, v_cache=FAKE, cache_seqlens=FAKE, k_new=None, v_new=None, seqlen_new=0,
+             cache_batch_idx=None, block_table=None, max_blocks_per_seq=0, cache_batch=8, cache_capacity=1024,
+             out=FAKE, lse=None, B=8, Hq=16, Hkv=4, Sq=3, D=128, softmax_scale=0.1, causal=1, window_left=-1,
+             window_right=-1, num_splits=0, workspace=FAKE, workspace_bytes=1 << 40, stream=S0)
+    a.update(kw)
+    return abi.fa_fwd_kvcache_ex(**a)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(k_new=FAKE), abi.FA_ERR_INVALID_ARG),                                  # k without v
+    (dict(k_new=FAKE, v_new=FAKE), abi.FA_ERR_INVALID_ARG),                      # new keys but seqlen_new = 0
+    (dict(seqlen_new=2), abi.FA_ERR_INVALID_ARG),                                # seqlen_new without k / v
+    (dict(block_table=FAKE, max_blocks_per_seq=4, cache_capacity=100), abi.FA_ERR_INVALID_ARG),  # page % 256
+    (dict(block_table=FAKE, max_blocks_per_seq=0, cache_capacity=256), abi.FA_ERR_INVALID_ARG),
+    (dict(block_table=FAKE, max_blocks_per_seq=4, cache_capacity=256, cache_batch_idx=FAKE), abi.FA_ERR_INVALID_ARG),
+    (dict(cache_batch=0), abi.FA_ERR_INVALID_ARG),
+    (dict(D=256), abi.FA_ERR_UNSUPPORTED),
+    (dict(workspace_bytes=0), abi.FA_ERR_WORKSPACE),
+    (dict(block_table=FAKE + 2, max_blocks_per_seq=4, cache_capacity=256), abi.FA_ERR_ALIGNMENT),
+])
+def test_kvcache_ex_argument_rules(lib, kw, want):
+    assert _kv_ex(**kw) == want
+
+
+def test_kvcache_ex_workspace_sizes(lib):
+    one = abi.fa_fwd_kvcache_ex_workspace_size(8, 16, 4, 1, 128, 4096, 0, 0)
+    four = abi.fa_fwd_kvcache_ex_workspace_size(8, 16, 4, 4, 128, 4096, 0, 0)
+    assert 0 < one < four                         # partials per query row
+    paged = abi.fa_fwd_kvcache_ex_workspace_size(8, 16, 4, 1, 128, 256, 16, 0)
+    assert paged == abi.fa_fwd_kvcache_ex_workspace_size(8, 16, 4, 1, 128, 4096, 0, 0)   # 16 pages of 256 keys
+    assert abi.fa_fwd_kvcache_ex_workspace_size(8, 16, 4, 1, 128, 100, 16, 0) == 0         # bad page size
+    assert abi.fa_fwd_kvcache_workspace_size(8, 16, 4, 1, 4096, 128, 0) == one
 
 
 def test_product_path_has_no_oracle_or_cpu_fallback():
