@@ -32,7 +32,7 @@ EXPORTS = (
     "fa_profile_begin", "fa_profile_read",
     "fa_fwd_kvcache_noalloc", "fa_fwd_kvcache_noalloc_scratch_bytes", "fa_debug_exp2_selftest",
     "fa_fwd_ex", "fa_bwd_ex", "fa_varlen_fwd_ex", "fa_varlen_bwd_ex",
-    "fa_fwd_kvcache_ex", "fa_fwd_kvcache_ex_workspace_size",
+    "fa_fwd_kvcache_ex", "fa_fwd_kvcache_ex_workspace_size", "fa_merge_lse",
 )
 
 FA_KERNEL_FWD = 0
@@ -71,6 +71,7 @@ _SIGS = {
     "fa_varlen_fwd_ex": (_I, [_P] * 7 + [_I] * 8 + [_F, _I, _I, _I, _P, _Z, _P]),
     "fa_varlen_bwd_ex": (_I, [_P] * 11 + [_I] * 8 + [_F, _I, _I, _I, _I, _P, _Z, _P]),
     "fa_fwd_kvcache_ex_workspace_size": (_Z, [_I] * 8),
+    "fa_merge_lse": (_I, [_P, _P] + [_I] * 6 + [_P, _P, _I, _P]),
     "fa_fwd_kvcache_ex": (_I, [_P] * 6 + [_I] + [_P] * 2 + [_I] * 3 + [_P] * 2 + [_I] * 5 + [_F] + [_I] * 4
                           + [_P, _Z, _P]),
 }
@@ -224,6 +225,11 @@ def fa_fwd_kvcache_ex(q, k_cache, v_cache, cache_seqlens, k_new, v_new, seqlen_n
                                     _ptr(lse), B, Hq, Hkv, Sq, D, float(softmax_scale), int(bool(causal)),
                                     int(window_left), int(window_right), int(num_splits), _ptr(workspace),
                                     workspace_bytes, _stream(stream))
+
+
+def fa_merge_lse(o_parts, lse_parts, num_parts, B, S, H, D, parts_fp32, out, lse, out_fp32, stream=None) -> int:
+    return load().fa_merge_lse(_ptr(o_parts), _ptr(lse_parts), int(num_parts), B, S, H, D, int(bool(parts_fp32)),
+                               _ptr(out), _ptr(lse), int(bool(out_fp32)), _stream(stream))
 
 
 def fa_get_device_status(stream=None) -> int:

@@ -157,6 +157,25 @@ def flash_attn_with_kvcache(q, k_cache, v_cache, cache_seqlens, softmax_scale=No
     return out, lse
 
 
+def merge_attention_parts(o_parts, lse_parts, out_dtype=torch.bfloat16, out=None):
+    """Merge results over disjoint key sets: o_parts (C, B, S, H, D) bf16 or fp32 and lse_parts (C, B, H, S)
+    fp32, as fa_fwd writes them per key set.  Returns (out (B, S, H, D), lse (B, H, S))."""
+    if o_parts.dtype not in (torch.bfloat16, torch.float32):
+        raise TypeError("o_parts must be bfloat16 or float32")
+    _check(o_parts, "o_parts", o_parts.dtype)
+    _check(lse_parts, "lse_parts", torch.float32)
+    C, B, S, H, D = o_parts.shape
+    if tuple(lse_parts.shape) != (C, B, H, S):
+        raise ValueError("lse_parts must be (C, B, H, S)")
+    if out is None:
+        out = torch.empty((B, S, H, D), dtype=out_dtype, device=o_parts.device)
+    _check(out, "out", out.dtype)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=o_parts.device)
+    _raise(abi.fa_merge_lse(o_parts, lse_parts, C, B, S, H, D, o_parts.dtype == torch.float32, out, lse,
+                            out.dtype == torch.float32), "fa_merge_lse")
+    return out, lse
+
+
 class FlashAttnFunction(torch.autograd.Function):
     """Autograd wrapper: forward = fa_fwd_ex, backward = fa_bwd_ex."""
 

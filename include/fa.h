@@ -238,6 +238,25 @@ FA_API int fa_fwd_kvcache_ex(const void* q, void* k_cache, void* v_cache, const 
                              float softmax_scale, int causal, int window_left, int window_right, int num_splits,
                              void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
+/* ------------------------------------------------------------------------- merging partial attention results
+ * fa_merge_lse: attention over the union of disjoint key sets from the results
+ * over each set (for context-parallel / ring attention, where each rank attends
+ * to one shard of the keys):
+ *     LSE = ln sum_c exp(LSE_c),   out = sum_c exp(LSE_c - LSE) O_c
+ * (README changelog 2.2: the split-KV decode merges its pieces the same way;
+ * the forward's LSE output is what makes it possible).  Parts with LSE_c = -inf
+ * contribute nothing; a row with every part empty gets out = 0, LSE = -inf.
+ *   o_parts   [num_parts, B, S, H, D], bf16 (parts_fp32 = 0) or float32 (1)
+ *   lse_parts [num_parts, B, H, S] float32 (the layout fa_fwd writes; a varlen
+ *             result [H, total] is B = 1, S = total)
+ *   out       [B, S, H, D], bf16 (out_fp32 = 0) or float32 (1)
+ *   lse       [B, H, S] float32, or NULL
+ * D in {64, 128, 256}.  out may be the memory of one of the parts (and lse of
+ * one of the LSE parts): each row is read completely before it is written.
+ */
+FA_API int fa_merge_lse(const void* o_parts, const float* lse_parts, int num_parts, int B, int S, int H, int D,
+                        int parts_fp32, void* out, float* lse, int out_fp32, fa_stream_t stream);
+
 /* ------------------------------------------------------------------------- KV-cache decode without caller memory
  * fa_fwd_kvcache_noalloc: the same computation as fa_fwd_kvcache, for callers
  * that cannot allocate device memory when they decode -- for example code that

@@ -178,3 +178,13 @@ def test_product_path_has_no_oracle_or_cpu_fallback():
             if f.endswith((".py", ".cu", ".cuh", ".h")):
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
+
+
+def test_merge_lse_argument_rules(lib):
+    ok = dict(o_parts=FAKE, lse_parts=FAKE, num_parts=2, B=1, S=8, H=2, D=128, parts_fp32=0, out=FAKE, lse=None,
+              out_fp32=0, stream=S0)
+    for kw, want in ((dict(o_parts=None), abi.FA_ERR_INVALID_ARG), (dict(num_parts=0), abi.FA_ERR_INVALID_ARG),
+                     (dict(D=96), abi.FA_ERR_UNSUPPORTED), (dict(out=FAKE + 4), abi.FA_ERR_ALIGNMENT)):
+        a = dict(ok)
+        a.update(kw)
+        assert abi.fa_merge_lse(**a) == want
