@@ -245,9 +245,12 @@ def run_ours(args, rank, world, local_rank):
     ff = fwd_flops(B, H, S, S, D, True)
     step_flops = 3.5 * ff
 
+    det = 1 if args.deterministic else 0
+
     def step():
         st = abi.fa_fwd(q, k, v, out, lse, B, H, H, S, S, D, scale, 1, None, 0, stream)
-        st |= abi.fa_bwd(q, k, v, out, do, lse, dq, dk, dv, B, H, H, S, S, D, scale, 1, ws, ws_bytes, stream)
+        st |= abi.fa_bwd_ex(q, k, v, out, do, lse, dq, dk, dv, B, H, H, S, S, D, scale, 1, -1, -1, det, ws, ws_bytes,
+                            stream)
         return st
 
     for _ in range(args.warmup):
@@ -281,6 +284,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     _, n_f, ms_f = abi.fa_profile_read(abi.FA_KERNEL_FWD)
     _, n_b, ms_b = abi.fa_profile_read(abi.FA_KERNEL_BWD)
+    _, n_q, ms_q = abi.fa_profile_read(abi.FA_KERNEL_BWD_DQ)   # deterministic backward only
     total_ms = max_over_ranks(total_ms, world, dev)
     if abi.fa_get_device_status() != 0:
         raise RuntimeError("a kernel reported a device-side timeout during the timed region")
@@ -298,7 +302,8 @@ def run_ours(args, rank, world, local_rank):
     def e2e_step():
         dq_ = {n: x.to(dev, non_blocking=True) for n, x in pin.items()}
         o_, l_ = A.flash_attn_func(dq_["q"], dq_["k"], dq_["v"], scale, True)
-        g = A.flash_attn_backward(dq_["do"], dq_["q"], dq_["k"], dq_["v"], o_, l_, scale, True)
+        g = A.flash_attn_backward(dq_["do"], dq_["q"], dq_["k"], dq_["v"], o_, l_, scale, True,
+                                  deterministic=bool(det))
         for n, x in zip(("out", "lse", "dq", "dk", "dv"), (o_, l_) + tuple(g)):
             host_out[n].copy_(x, non_blocking=True)
 
@@ -323,18 +328,21 @@ def run_ours(args, rank, world, local_rank):
     if rank != 0:
         return 0
     peak_t = pk["bf16_tflops"]
-    bwd_ms = ms_b / max(n_b, 1)
+    bwd_ms = ms_b / max(n_b, 1) + (ms_q / max(n_q, 1) if det else 0.0)
     fwd_ms = ms_f / max(n_f, 1)
     bwd_tf = 2.5 * ff / (bwd_ms * 1e-3) / 1e12
     fwd_tf = ff / (fwd_ms * 1e-3) / 1e12
-    traffic = traffic_record("bwd_kernel", "exact_tiled_attention_41_b200/csrc/bwd.cu")
+    traffic = None if det else traffic_record("bwd_kernel", "exact_tiled_attention_41_b200/csrc/bwd.cu")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(WORKLOAD, global_batch=4 * world, parallelism="replicas" if world > 1 else "single",
-                       l2="flushed before every step (256 MiB write, outside the per-step events)"),
-        "roofline": {"bound": "tensor", "kernel": "bwd_kernel (backward main)", "achieved": bwd_tf,
+                       l2="flushed before every step (256 MiB write, outside the per-step events)",
+                       **({"backward": "deterministic"} if det else {})),
+        "roofline": {"bound": "tensor",
+                     "kernel": "bwd_kernel + dq_kernel (deterministic backward)" if det else "bwd_kernel (backward main)",
+                     "achieved": bwd_tf,
                      "peak": peak_t, "unit": "TFLOP/s", "frac": bwd_tf / peak_t, "traffic": traffic,
                      "peak_source": f"{pk_kind} bf16_tflops (burst)",
                      "algorithmic_flops_per_launch": 2.5 * ff, "avg_launch_ms": bwd_ms, "launches": n_b},
@@ -457,7 +465,54 @@ def measure_extras(torch, abi, A, W, dev, pk):
         "ms": dms, "gbs": alg_bytes / dms / 1e6, "frac_of_measured_hbm": alg_bytes / dms / 1e6 / pk["hbm_gbs"],
         "split_kernel_ms": split_ms, "split_kernel_gbs": kv_bytes / split_ms / 1e6,
         "algorithmic_bytes": alg_bytes}
-    del t, w
+
+    # the same cache in pages of 256 keys behind a random block table
+    page = 256
+    nps = cap // page
+    gperm = torch.Generator("cpu").manual_seed(1)
+    table = torch.randperm(B * nps, generator=gperm).reshape(B, nps).to(torch.int32).to(dev)
+    kp = torch.empty((B * nps, page, Hkv, D), dtype=torch.bfloat16, device=dev)
+    vp = torch.empty_like(kp)
+    kp[table.flatten().long()] = t["k_cache"].view(B * nps, page, Hkv, D)
+    vp[table.flatten().long()] = t["v_cache"].view(B * nps, page, Hkv, D)
+    del t["k_cache"], t["v_cache"]
+    nbp = abi.fa_fwd_kvcache_ex_workspace_size(B, Hq, Hkv, 1, D, page, nps, 0)
+    wsp = torch.empty(nbp, dtype=torch.uint8, device=dev)
+    pms = timed(lambda: abi.fa_fwd_kvcache_ex(t["q"], kp, vp, lens, None, None, 0, None, table, nps, B * nps, page,
+                                              out, lse, B, Hq, Hkv, 1, D, w.scale, 0, -1, -1, 0, wsp, nbp, stream), 10)
+    res["decode_paged256_B64_Hq32_Hkv8_cap16384_D128"] = {
+        "ms": pms, "gbs": alg_bytes / pms / 1e6, "frac_of_measured_hbm": alg_bytes / pms / 1e6 / pk["hbm_gbs"]}
+
+    # four new tokens per row (speculative-decoding shape), appended in place, causal
+    sn = 4
+    g4 = torch.Generator(str(dev)).manual_seed(2)
+    q4 = torch.randn((B, sn, Hq, D), generator=g4, device=dev).to(torch.bfloat16)
+    kn = torch.randn((B, sn, Hkv, D), generator=g4, device=dev).to(torch.bfloat16)
+    vn = torch.randn((B, sn, Hkv, D), generator=g4, device=dev).to(torch.bfloat16)
+    lens4 = torch.clamp(lens, max=cap - sn)
+    out4 = torch.empty_like(q4)
+    lse4 = torch.empty((B, Hq, sn), dtype=torch.float32, device=dev)
+    nb4 = abi.fa_fwd_kvcache_ex_workspace_size(B, Hq, Hkv, sn, D, page, nps, 0)
+    ws4 = torch.empty(nb4, dtype=torch.uint8, device=dev)
+    ams = timed(lambda: abi.fa_fwd_kvcache_ex(q4, kp, vp, lens4, kn, vn, sn, None, table, nps, B * nps, page, out4,
+                                              lse4, B, Hq, Hkv, sn, D, w.scale, 1, -1, -1, 0, ws4, nb4, stream), 10)
+    a_bytes = (float(lens4.sum().item()) + B * sn) * Hkv * D * 2 * 2 + 2 * q4.numel() * 2 + 2 * kn.numel() * 2 * 2
+    res["decode_append4_causal_paged256_B64_Hq32_Hkv8_D128"] = {
+        "ms": ams, "gbs": a_bytes / ams / 1e6, "frac_of_measured_hbm": a_bytes / ams / 1e6 / pk["hbm_gbs"]}
+    del t, w, kp, vp, wsp, ws4
+
+    # merging four partial results of the long-context GQA output (B=2, S=8192, H=32, D=128, bf16)
+    C, Bm, Sm, Hm, Dm = 4, 2, 8192, 32, 128
+    gm = torch.Generator(str(dev)).manual_seed(3)
+    o_parts = torch.randn((C, Bm, Sm, Hm, Dm), generator=gm, device=dev).to(torch.bfloat16)
+    l_parts = torch.randn((C, Bm, Hm, Sm), generator=gm, device=dev)
+    o_m = torch.empty((Bm, Sm, Hm, Dm), dtype=torch.bfloat16, device=dev)
+    l_m = torch.empty((Bm, Hm, Sm), dtype=torch.float32, device=dev)
+    mms = timed(lambda: abi.fa_merge_lse(o_parts, l_parts, C, Bm, Sm, Hm, Dm, 0, o_m, l_m, 0, stream), 10)
+    m_bytes = (C + 1) * (o_m.numel() * 2 + l_m.numel() * 4)
+    res["merge_lse_4parts_B2_S8192_H32_D128"] = {
+        "ms": mms, "gbs": m_bytes / mms / 1e6, "frac_of_measured_hbm": m_bytes / mms / 1e6 / pk["hbm_gbs"]}
+    del o_parts, l_parts, o_m, l_m
     torch.cuda.empty_cache()
     return res
 
@@ -469,6 +524,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="time the step with the deterministic backward (dq from the query-tile-stationary pass)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     args = ap.parse_args()

@@ -450,7 +450,9 @@ static int run_dq(const Problem& pr, const void* dout, const float* lse2, const 
         attr_set[dev.id & 63] = true;
     }
     const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
+    prof_before(3, stream);
     kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mdo, mk, mv, p);
+    prof_after(3, stream);
     return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
 }
 

@@ -305,15 +305,16 @@ FA_API unsigned long long fa_set_wait_timeout_ns(unsigned long long ns);
 
 /* Kernel timing with CUDA events, for benchmarks.  fa_profile_begin(1) makes
  * every later launch of the main kernel of fa_fwd / fa_varlen_fwd (id 0), the
- * main backward kernel of fa_bwd / fa_varlen_bwd (id 1) and the split kernel of
- * fa_fwd_kvcache (id 2) record a pair of CUDA events around itself on the
+ * main backward kernel of fa_bwd / fa_varlen_bwd (id 1), the split kernel of
+ * fa_fwd_kvcache (id 2) and the dQ pass of the deterministic backward (id 3)
+ * record a pair of CUDA events around itself on the
  * launching stream (up to 1024 launches per id; later ones are not recorded),
  * and clears earlier records; fa_profile_begin(0) stops recording.
  * fa_profile_read, after the caller has synchronised those streams, returns the
  * number of recorded launches of `kernel_id` and the sum of their durations in
  * milliseconds.  Events are created on first use; no device memory is allocated.
  */
-enum fa_kernel_id { FA_KERNEL_FWD = 0, FA_KERNEL_BWD = 1, FA_KERNEL_DECODE = 2 };
+enum fa_kernel_id { FA_KERNEL_FWD = 0, FA_KERNEL_BWD = 1, FA_KERNEL_DECODE = 2, FA_KERNEL_BWD_DQ = 3 };
 FA_API int fa_profile_begin(int enable);
 FA_API int fa_profile_read(int kernel_id, int* launches, float* total_ms);
 
