@@ -18,8 +18,9 @@
 //      tile (causal masks and sliding windows cut the range at both ends).  Roles (16 warps, registers redistributed with setmaxnreg):
 //        warps 0-7   two compute warpgroups, thread = key row, each owning 64 of
 //                    the 128 query columns: P^T, dS^T from S^T and dP^T in tensor
-//                    memory (written back as bf16, dS^T also to shared memory);
-//                    dV (warpgroup 0) / dK (warpgroup 1) epilogue
+//                    memory, both written back as bf16 into the warpgroup's own 64
+//                    columns of S^T (dS^T also to shared memory), so dP^T's columns
+//                    are free for dQ; dV (warpgroup 0) / dK (warpgroup 1) epilogue
 //        warps 8-11  dQ: thread = query row; reads the dQ tile from tensor memory
 //                    and adds it to the fp32 accumulator (vector atomics); each half
 //                    of the tile is released as soon as it is in registers, so the
@@ -28,10 +29,12 @@
 //        warp 12     producer: K, V once per unit; Q, dO tiles (TMA) and the
 //                    tile's LSE2 / Delta (plain loads) through a 2-stage ring
 //        warp 13     tensor memory and every tcgen05 MMA, in this order per tile:
-//                    S^T = K Q^T, dP^T = V dO^T              (K-major x K-major)
-//                    dQ = dS K into the columns of S^T / dP^T left free by the
-//                    bf16 P^T / dS^T, so the dQ read-out overlaps   (N-major x N-major)
-//                    dV += P^T dO, dK += dS^T Q               (tensor-memory A)
+//                    S^T = K Q^T, then dP^T = V dO^T once the previous dQ read-out
+//                    released dP^T's columns (K-major x K-major); dV += P^T dO,
+//                    dK += dS^T Q over queries 0-63 as soon as warpgroup 0 is done
+//                    (tensor-memory A), while warpgroup 1 still works; then
+//                    dQ = dS K, all D columns in one product, into dP^T's columns,
+//                    so the dQ read-out overlaps the dV, dK products over queries 64-127
 //   3. convert: dQ = bf16(scale * dQacc).
 // The deterministic backward runs the main kernel with DQ = false (no dQ product,
 // no reduce-adds, warps 8-11 idle) and computes dq in the query-tile-stationary
@@ -116,18 +119,24 @@ struct BwdCfg {
     static constexpr uint32_t OFF_K = 0, OFF_V = T_BYTES, OFF_Q = 2 * T_BYTES, OFF_DO = (2 + ST) * T_BYTES,
                               OFF_DS = (2 + 2 * ST) * T_BYTES, OFF_STAT = OFF_DS + DS_BYTES,
                               OFF_BAR = OFF_STAT + 2 * ST * 128 * 4;
-    static constexpr int NUM_BARS = 2 + 2 * ST + 6;
+    static constexpr int NUM_BARS = 2 + 2 * ST + 7;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
-    // tensor memory: dV | dK | S^T | dP^T.  After the gradient step P^T and dS^T (bf16) occupy the
-    // low 64 columns of S^T and dP^T; dQ (fp32) is accumulated into their free high 64 columns.
-    static constexpr uint32_t COL_DV = 0, COL_DK = D, COL_S = 2 * D, COL_DP = 2 * D + 128;
-    static constexpr uint32_t COL_DQ(int h) { return h == 0 ? COL_S + 64 : COL_DP + 64; }
+    // tensor memory: dV | dK | S^T | dP^T.  After the gradient step the packed bf16 P^T and dS^T of each
+    // 32-query half sit in that half's own 32 columns of S^T; dQ (fp32, D columns) is accumulated over
+    // dP^T, whose values the warpgroups have read by then.
+    static constexpr uint32_t COL_DV = 0, COL_DK = D, COL_S = 2 * D, COL_DP = 2 * D + 128, COL_DQ = COL_DP;
+    // packed P^T / dS^T of queries [16 kk, 16 kk + 16): query half (kk >> 1) of 32 lives in columns
+    // [32 (kk >> 1), +32) of S^T, P^T first, dS^T 16 columns later
+    static constexpr uint32_t COL_P(int kk) { return COL_S + (kk >> 1) * 32 + (kk & 1) * 8; }
+    static constexpr uint32_t COL_DSP(int kk) { return COL_P(kk) + 16; }
     static_assert(2 * D + 256 <= 512, "tensor memory budget");
-    static_assert(D == 64 || D == 128, "dQ halves map onto the free columns for D <= 128");
+    static_assert(D == 64 || D == 128, "dQ fits dP^T's 128 columns for D <= 128");
     // 16 warps: 0-7 two compute warpgroups (query columns 0-63 / 64-127), 8-11 dQ warpgroup,
     // 12 producer, 13 MMA issuer, 14-15 idle.  Registers: launch at 128 per thread (512 x 128 = 65536);
-    // 2 x 128 x 184 + 128 x 64 + 128 x 72 = 64512.  The host checks the launch count.
-    static constexpr int THREADS = 512, LAUNCH_REGS = 128, COMPUTE_REGS = 184, DQ_REGS = 64, OTHER_REGS = 72;
+    // the producer / MMA warpgroup gives 40 per thread to the dQ warpgroup, which holds a whole dQ row:
+    // 2 x 128 x 128 + 128 x 168 + 128 x 88 = 65536.  The host checks the launch count.
+    static constexpr int THREADS = 512, LAUNCH_REGS = 128, COMPUTE_REGS = 128, DQ_REGS = 168, OTHER_REGS = 88;
+    static_assert(COMPUTE_REGS == LAUNCH_REGS, "the compute warpgroups keep the launch count");
     static_assert(2 * 128 * COMPUTE_REGS + 128 * DQ_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
@@ -148,8 +157,9 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t kv_full = b0, kv_empty = b0 + 8;
     auto q_full = [&](int s) { return b0 + 8u * (2 + s); };
     auto q_empty = [&](int s) { return b0 + 8u * (2 + ST + s); };
+    // p_full / p_full_hi: compute warpgroup 0 (query columns 0-63) / 1 (64-127) done
     const uint32_t s_full = b0 + 8u * (2 + 2 * ST), p_full = s_full + 8, dq_full = s_full + 16,
-                   dq_empty = s_full + 24, dkv_full = s_full + 32, dq_empty_hi = s_full + 40;
+                   dq_empty = s_full + 24, dkv_full = s_full + 32, dq_empty_hi = s_full + 40, p_full_hi = s_full + 48;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PRODUCER = 12, MMA = 13;
@@ -166,11 +176,12 @@ __global__ void __launch_bounds__(512, 1)
             mbar_init(bars + 2 + ST + s, 1);
         }
         mbar_init(bars + 2 + 2 * ST + 0, 1);    // s_full
-        mbar_init(bars + 2 + 2 * ST + 1, 256);  // p_full: both compute warpgroups
+        mbar_init(bars + 2 + 2 * ST + 1, 128);  // p_full: compute warpgroup 0 (query columns 0-63)
         mbar_init(bars + 2 + 2 * ST + 2, 1);    // dq_full
         mbar_init(bars + 2 + 2 * ST + 3, 128);  // dq_empty: dQ columns in the S^T region read out
         mbar_init(bars + 2 + 2 * ST + 4, 1);    // dkv_full
         mbar_init(bars + 2 + 2 * ST + 5, 128);  // dq_empty_hi: dQ columns in the dP^T region read out
+        mbar_init(bars + 2 + 2 * ST + 6, 128);  // p_full_hi: compute warpgroup 1 (query columns 64-127)
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -248,7 +259,7 @@ __global__ void __launch_bounds__(512, 1)
             if (lane == 0) {
                 constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
                 constexpr uint32_t id_tn = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
-                constexpr uint32_t id_dq = idesc_bf16_f32(128, 64, true, true);      // dQ, 64 columns at a time
+                constexpr uint32_t id_dq = idesc_bf16_f32(128, D, true, true);       // dQ, all D columns
                 uint32_t unit_it = 0, q_it = 0, g_it = 0;
                 bool ok = true;
                 for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
@@ -259,7 +270,6 @@ __global__ void __launch_bounds__(512, 1)
                     for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
                         const int st = q_it % ST;
                         if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
-                        if (DQ && g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
                         tc_fence_after();
                         const uint8_t* sq = smem + C::OFF_Q + st * C::T_BYTES;
                         const uint8_t* sdo = smem + C::OFF_DO + st * C::T_BYTES;
@@ -269,7 +279,8 @@ __global__ void __launch_bounds__(512, 1)
                             umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + o), 16, 1024),
                                     sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
                         }
-                        // the previous tile's dQ columns in the dP^T region must be read out first
+                        // dP^T goes where the previous tile's dQ was: both halves of it must be read out
+                        if (DQ && g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
                         if (DQ && g_it > 0 && !mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
@@ -279,30 +290,37 @@ __global__ void __launch_bounds__(512, 1)
                                     sdesc_sw128(smem_u32(sdo + o), 16, 1024), id_kk, kk > 0);
                         }
                         umma_commit(s_full);
+                        // dV += P^T dO, dK += dS^T Q over queries 0-63, as soon as warpgroup 0 is done
                         if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
+                            umma_ts(tmem + C::COL_DV, tmem + C::COL_P(kk),
+                                    sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DSP(kk),
+                                    sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                        }
+                        if (!mbar_wait(p_full_hi, g_it & 1, w)) { ok = false; break; }
+                        tc_fence_after();
                         if constexpr (DQ) {
-                            // dQ = dS K first, into the free high columns, so its read-out overlaps dV / dK
+                            // dQ = dS K over dP^T's columns (read out by the dQ warpgroup while dV / dK finish)
 #pragma unroll
-                            for (int hh = 0; hh < D / 64; ++hh) {
-#pragma unroll
-                                for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
-                                    umma_ss(tmem + C::COL_DQ(hh),
-                                            sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
-                                            sdesc_sw128(smem_u32(smem + C::OFF_K + hh * 128 * 128 + kk * 16 * 128),
-                                                        128 * 128, 1024),
-                                            id_dq, kk > 0);
-                                }
+                            for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
+                                umma_ss(tmem + C::COL_DQ,
+                                        sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
+                                        sdesc_sw128(smem_u32(smem + C::OFF_K + kk * 16 * 128), 128 * 128, 1024),
+                                        id_dq, kk > 0);
                             }
                             umma_commit(dq_full);
                         }
+                        // dV, dK over queries 64-127
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 query rows
-                            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                            umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8,
-                                    sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
-                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8,
-                                    sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                        for (int kk = 4; kk < 8; ++kk) {
+                            umma_ts(tmem + C::COL_DV, tmem + C::COL_P(kk),
+                                    sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, 1u);
+                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DSP(kk),
+                                    sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, 1u);
                         }
                         umma_commit(q_empty(st));
                     }
@@ -315,7 +333,7 @@ __global__ void __launch_bounds__(512, 1)
             __syncwarp();
         }
     } else if (warp >= 8) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::DQ_REGS));
+        if constexpr (DQ) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::DQ_REGS));
         // ------------------------------------------------------------ dQ warpgroup (thread = query row)
         if constexpr (DQ) {
         const int wq = warp - 8;
@@ -336,31 +354,29 @@ __global__ void __launch_bounds__(512, 1)
                 if (!mbar_wait(dq_full, g_it & 1, w)) { ok = false; break; }
                 tc_fence_after();
                 float4* acc = reinterpret_cast<float4*>(p.dq_acc) + static_cast<size_t>(h) * (D / 4) * p.Tq + tok;
-#pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t ra[32];
-                    tmem_ld32(tmem + lb + C::COL_DQ(cc >> 1) + (cc & 1) * 32, ra);
-                    tmem_ld_wait_tie(ra);
-                    // release each half of the tile as soon as it sits in registers: the next S^T
-                    // overwrites the first half, the next dP^T the second
-                    if (cc == 1 || cc == D / 32 - 1) {
-                        tc_fence_before();
-                        if (cc == 1) mbar_arrive(dq_empty);
-                        if (cc == D / 32 - 1) mbar_arrive(dq_empty_hi);
-                    }
-                    if (valid) {
+                // the whole dQ row in registers at once, so its columns are released before the reduce-adds
+                uint32_t ra[D / 32][32];
+#pragma unroll
+                for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tmem + lb + C::COL_DQ + cc * 32, ra[cc]);
+                tmem_ld_wait_tie(ra[0]);
+#pragma unroll
+                for (int cc = 1; cc < D / 32; ++cc) reg_tie(ra[cc]);
+                tc_fence_before();
+                mbar_arrive(dq_empty);
+                mbar_arrive(dq_empty_hi);
+                if (valid) {
+#pragma unroll
+                    for (int cc = 0; cc < D / 32; ++cc)
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
                             atomicAdd(acc + static_cast<size_t>(cc * 8 + e) * p.Tq,
-                                      make_float4(__uint_as_float(ra[4 * e]), __uint_as_float(ra[4 * e + 1]),
-                                                  __uint_as_float(ra[4 * e + 2]), __uint_as_float(ra[4 * e + 3])));
-                    }
+                                      make_float4(__uint_as_float(ra[cc][4 * e]), __uint_as_float(ra[cc][4 * e + 1]),
+                                                  __uint_as_float(ra[cc][4 * e + 2]), __uint_as_float(ra[cc][4 * e + 3])));
                 }
             }
         }
         }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
         // ------------------------------------------------------------ compute warpgroups (thread = key row)
         const int gq = warp >> 2;                  // query columns [64 gq, 64 gq + 64)
         const int r = (warp & 3) * 32 + lane;
@@ -392,33 +408,11 @@ __global__ void __launch_bounds__(512, 1)
             for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
                 const int m0 = (t.m_start + it % t.n_m) * 128;
                 const int st = q_it % ST;
+                // the statistics arrive with the Q / dO tile
                 bool got = mbar_wait(s_full, g_it & 1, w);
                 got = got && mbar_wait(q_full(st), (q_it / ST) & 1, w);
-                uint32_t sa[2][32], da[2][32];
-                if (__all_sync(0xffffffffu, got)) {
-                    tc_fence_after();
-                    tmem_ld32(tmem + lb + C::COL_S + 64 * gq, sa[0]);
-                    tmem_ld32(tmem + lb + C::COL_S + 64 * gq + 32, sa[1]);
-                    tmem_ld32(tmem + lb + C::COL_DP + 64 * gq, da[0]);
-                    tmem_ld32(tmem + lb + C::COL_DP + 64 * gq + 32, da[1]);
-                    tmem_ld_wait_tie(sa[0]);
-                    reg_tie(sa[1]);
-                    reg_tie(da[0]);
-                    reg_tie(da[1]);
-                } else {
-                    got = false;
-                }
-                // Both warpgroups hold their columns before either overwrites the low columns with
-                // P^T / dS^T.  Every compute thread passes this barrier once per iteration, also on abort,
-                // and all of them leave together if any wait gave up.
-                uint32_t all_got;
-                asm volatile(
-                    "{\n\t.reg .pred pa, pb;\n\tsetp.ne.u32 pa, %1, 0;\n\t"
-                    "bar.red.and.pred pb, 1, 256, pa;\n\tselp.u32 %0, 1, 0, pb;\n\t}\n"
-                    : "=r"(all_got)
-                    : "r"(static_cast<uint32_t>(got))
-                    : "memory");
-                if (!all_got) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
                 // allowed local query columns of this tile: qmin .. qmax
                 const int qmin = q_lo - m0, qmax = q_hi - m0;
                 const bool full_row = qmin <= 64 * gq && qmax >= 64 * gq + 63;
@@ -427,8 +421,14 @@ __global__ void __launch_bounds__(512, 1)
                 const float* del_t = sDel + st * 128 + 64 * gq;
                 const float2 c2v = make_float2(c2, c2);
                 uint8_t* ds_row = smem + C::OFF_DS + gq * 128 * 128 + r * 128;
+                // the two 32-column halves one after the other, so only one half's values are live
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
+                    uint32_t sh[32], dh[32];
+                    tmem_ld32(tmem + lb + C::COL_S + 64 * gq + 32 * half, sh);
+                    tmem_ld32(tmem + lb + C::COL_DP + 64 * gq + 32 * half, dh);
+                    tmem_ld_wait_tie(sh);
+                    reg_tie(dh);
                     uint32_t pp[16], dd[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 4) {
@@ -438,8 +438,8 @@ __global__ void __launch_bounds__(512, 1)
                         for (int x = 0; x < 4; x += 2) {
                             const float la = x == 0 ? l4.x : l4.z, lbv = x == 0 ? l4.y : l4.w;
                             const float dla = x == 0 ? d4.x : d4.z, dlb = x == 0 ? d4.y : d4.w;
-                            const float2 sv = make_float2(__uint_as_float(sa[half][e + x]), __uint_as_float(sa[half][e + x + 1]));
-                            const float2 dv = make_float2(__uint_as_float(da[half][e + x]), __uint_as_float(da[half][e + x + 1]));
+                            const float2 sv = make_float2(__uint_as_float(sh[e + x]), __uint_as_float(sh[e + x + 1]));
+                            const float2 dv = make_float2(__uint_as_float(dh[e + x]), __uint_as_float(dh[e + x + 1]));
                             const float2 a = ffma2(sv, c2v, make_float2(-la, -lbv));
                             float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
                             if (any_mask) {
@@ -452,9 +452,10 @@ __global__ void __launch_bounds__(512, 1)
                             dd[(e + x) / 2] = pack_bf16x2(ds.x, ds.y);
                         }
                     }
-                    // P^T and dS^T of query columns [64 gq + 32 half, +32) -> packed columns [32 gq + 16 half, +16)
-                    tmem_st16(tmem + lb + C::COL_S + 32 * gq + 16 * half, pp);
-                    tmem_st16(tmem + lb + C::COL_DP + 32 * gq + 16 * half, dd);
+                    // P^T, dS^T of query columns [64 gq + 32 half, +32) -> packed S^T columns
+                    // [64 gq + 32 half, +16) and [64 gq + 32 half + 16, +16): the columns just read
+                    tmem_st16(tmem + lb + C::COL_S + 64 * gq + 32 * half, pp);
+                    tmem_st16(tmem + lb + C::COL_S + 64 * gq + 32 * half + 16, dd);
 #pragma unroll
                     for (int q4 = 0; q4 < 4; ++q4) {
                         const int cin = half * 4 + q4;            // 16-byte chunk of the 64-query box row
@@ -465,7 +466,7 @@ __global__ void __launch_bounds__(512, 1)
                 tmem_st_wait();
                 fence_proxy_async_smem();
                 tc_fence_before();
-                mbar_arrive(p_full);
+                mbar_arrive(gq == 0 ? p_full : p_full_hi);
             }
             if (!ok) break;
             // -------------------------------------------------- epilogue: warpgroup 0 writes dV, 1 writes dK
