@@ -509,6 +509,352 @@ __global__ void __launch_bounds__(512, 1)
     }
 }
 
+// ---------------------------------------------------------------------------- two items in flight (D = 128, no dQ)
+// The main kernel of the deterministic backward at head dim 128 (dQ comes from the query-tile-stationary
+// pass of bwd_dq.cu), with query items of 64 rows and two tensor-memory buffers, so that the gradient step
+// of one item overlaps the tensor-core work of the next:
+//   tensor memory: dV [0,128) | dK [128,256) | buffer 0 [256,384) | buffer 1 [384,512),
+//   buffer b = S^T (64 columns) | dP^T (64 columns); item i uses buffer i % 2.
+// Items alternate between the two compute warpgroups (warpgroup b takes the items of buffer b, the low /
+// high 64 query rows of every 128-row query tile).  Per item the MMA warp issues S^T, dP^T of item i,
+// then dV += P^T dO, dK += dS^T Q of item i - 1, so the tensor core works on one item while a warpgroup
+// works on the other.  A warpgroup packs P^T and dS^T (bf16 pairs) into the 32-column halves of S^T it
+// has just read.  Measured on B200 this beats the one-item-at-a-time kernel only without the dQ product:
+// with it, the 64-query products read K, V and K^T from shared memory twice per 128-row tile and the
+// tensor pipe, not the gradient step, sets the pace.
+struct PPCfg {
+    static constexpr int D = 128;
+    static constexpr int ST = 3;                                 // Q / dO item stages
+    static constexpr uint32_t KV_BYTES = 128 * D * 2;            // K or V tile: two [128 x 64] boxes
+    static constexpr uint32_t IT_BYTES = 64 * D * 2;             // Q or dO item: two [64 x 64] boxes
+    static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_Q = 2 * KV_BYTES, OFF_DO = OFF_Q + ST * IT_BYTES,
+                              OFF_STAT = OFF_DO + ST * IT_BYTES, OFF_BAR = OFF_STAT + 2 * ST * 64 * 4;
+    // kv_full, kv_empty, q_full[ST], q_empty[ST], s_full[2], p_full[2], dkv_full, dkv_empty
+    static constexpr int NUM_BARS = 2 + 2 * ST + 4 + 2;
+    static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr uint32_t COL_DV = 0, COL_DK = 128;
+    static constexpr uint32_t COL_S(int b) { return 256 + 128 * b; }
+    static constexpr uint32_t COL_DP(int b) { return 256 + 128 * b + 64; }
+    // packed P^T / dS^T of item queries [16 kk, 16 kk + 16): in the 32-column half (kk >> 1) of S^T
+    static constexpr uint32_t COL_P(int b, int kk) { return COL_S(b) + (kk >> 1) * 32 + (kk & 1) * 8; }
+    static constexpr uint32_t COL_DSP(int b, int kk) { return COL_P(b, kk) + 16; }
+    // 12 warps: 0-3 / 4-7 compute warpgroups 0 / 1, 8 producer, 9 MMA, 10-11 idle
+    static constexpr int THREADS = 384, LAUNCH_REGS = 168, COMPUTE_REGS = 200, OTHER_REGS = 96;
+    static_assert(2 * 128 * COMPUTE_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+__global__ void __launch_bounds__(384, 1)
+    bwd_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const __grid_constant__ BwdParams p) {
+    using C = PPCfg;
+    constexpr int D = C::D;
+    constexpr int ST = C::ST;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);          // [ST][64]
+    float* sDel = sLSE + ST * 64;                                        // [ST][64]
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    const uint32_t b0 = smem_u32(bars);
+    const uint32_t kv_full = b0, kv_empty = b0 + 8;
+    auto q_full = [&](int s) { return b0 + 8u * (2 + s); };
+    auto q_empty = [&](int s) { return b0 + 8u * (2 + ST + s); };
+    const uint32_t bb = b0 + 8u * (2 + 2 * ST);
+    auto s_full = [&](int b) { return bb + 8u * b; };
+    auto p_full = [&](int b) { return bb + 16 + 8u * b; };
+    const uint32_t dkv_full = bb + 32, dkv_empty = bb + 40;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    constexpr int PRODUCER = 8, MMA = 9;
+
+    if ((smem_u32(smem) & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
+        if (threadIdx.x == 0) atomicCAS(p.status, 0, 2);
+        return;
+    }
+    if (threadIdx.x == 0) {
+        mbar_init(bars + 0, 1);
+        mbar_init(bars + 1, 1);
+        for (int s = 0; s < ST; ++s) {
+            mbar_init(bars + 2 + s, 33);        // 32 producer lanes (statistics) + the TMA expect-tx arrival
+            mbar_init(bars + 2 + ST + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(bars + 2 + 2 * ST + b, 1);        // s_full[b]
+            mbar_init(bars + 2 + 2 * ST + 2 + b, 128);  // p_full[b]: compute warpgroup b
+        }
+        mbar_init(bars + 2 + 2 * ST + 4, 1);            // dkv_full
+        mbar_init(bars + 2 + 2 * ST + 5, 256);          // dkv_empty: both epilogues read dV / dK
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == PRODUCER && lane == 0) {
+        tma_prefetch_map(&tmQ);
+        tma_prefetch_map(&tmK);
+        tma_prefetch_map(&tmV);
+        tma_prefetch_map(&tmDO);
+    }
+    if (warp == MMA) {
+        tmem_alloc(smem_u32(tmem_slot), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const Watch w{abort_flag, p.status, p.timeout_ns};
+    const int G = p.group;
+
+    if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
+        if (warp == PRODUCER) {
+            // -------------------------------------------------------- producer (whole warp)
+            uint32_t unit_it = 0, q_it = 0;
+            bool ok = true;
+            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+                if (u >= p.num_units) continue;
+                const BUnit t = decode_bunit(p, u);
+                if (t.skip || t.n_it == 0) continue;
+                if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(kv_full, 2 * C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c) {
+                        tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
+                        tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
+                    }
+                }
+                ++unit_it;
+                for (int it = 0; it < t.n_it && ok; ++it) {
+                    const int h = t.hk * G + it / t.n_m;
+                    for (int qh = 0; qh < 2; ++qh, ++q_it) {
+                        const int row0 = (t.m_start + it % t.n_m) * 128 + 64 * qh;
+                        const int st = q_it % ST;
+                        if (q_it >= ST && !mbar_wait(q_empty(st), ((q_it / ST) - 1) & 1, w)) { ok = false; break; }
+                        // item statistics; rows past the sequence get LSE2 = +inf (P = 0) and Delta = 0
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const int qi = lane * 2 + e;
+                            const int row = row0 + qi;
+                            const bool in = row < t.Lq;
+                            const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
+                            sLSE[st * 64 + qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
+                            sDel[st * 64 + qi] = in ? __ldg(p.delta + idx) : 0.f;
+                        }
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(q_full(st), 2 * C::IT_BYTES);
+#pragma unroll
+                            for (int c = 0; c < D / 64; ++c) {
+                                tma_load_3d(smem_u32(smem + C::OFF_Q + st * C::IT_BYTES + c * 64 * 128), &tmQ,
+                                            q_full(st), c * 64, h, t.q_start + row0);
+                                tma_load_3d(smem_u32(smem + C::OFF_DO + st * C::IT_BYTES + c * 64 * 128), &tmDO,
+                                            q_full(st), c * 64, h, t.q_start + row0);
+                            }
+                        }
+                        mbar_arrive(q_full(st));
+                    }
+                }
+            }
+            __syncwarp();
+        } else if (warp == MMA) {
+            // -------------------------------------------------------- MMA issuer
+            if (lane == 0) {
+                constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);    // S^T, dP^T of an item
+                constexpr uint32_t id_t = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
+                uint32_t unit_it = 0, q_it = 0, gi = 0;
+                bool ok = true;
+                // dV, dK of item g (buffer g % 2, stage st); `first`: the unit's first item overwrites dV, dK
+                auto post = [&](uint32_t g, int st, bool first) -> bool {
+                    const int b = g & 1;
+                    if (!mbar_wait(p_full(b), (g >> 1) & 1, w)) return false;
+                    // the previous unit's epilogues must have read dV and dK before they are overwritten
+                    if (first && unit_it > 0 && !mbar_wait(dkv_empty, (unit_it - 1) & 1, w)) return false;
+                    tc_fence_after();
+                    const uint8_t* sq = smem + C::OFF_Q + st * C::IT_BYTES;
+                    const uint8_t* sdo = smem + C::OFF_DO + st * C::IT_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {     // K-dim = 64 item queries
+                        const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
+                        umma_ts(tmem + C::COL_DV, tmem + C::COL_P(b, kk),
+                                sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 64 * 128, 1024), id_t, acc);
+                        umma_ts(tmem + C::COL_DK, tmem + C::COL_DSP(b, kk),
+                                sdesc_sw128(smem_u32(sq + kk * 16 * 128), 64 * 128, 1024), id_t, acc);
+                    }
+                    umma_commit(q_empty(st));
+                    return true;
+                };
+                for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+                    if (u >= p.num_units) continue;
+                    const BUnit t = decode_bunit(p, u);
+                    if (t.skip || t.n_it == 0) continue;
+                    if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
+                    const int items = 2 * t.n_it;
+                    uint32_t prev_g = 0;
+                    int prev_st = 0;
+                    for (int i = 0; i < items; ++i, ++q_it, ++gi) {
+                        const int st = q_it % ST;
+                        const int b = gi & 1;
+                        if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint8_t* sq = smem + C::OFF_Q + st * C::IT_BYTES;
+                        const uint8_t* sdo = smem + C::OFF_DO + st * C::IT_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oa = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+                            const uint32_t ob = (kk >> 2) * 64 * 128 + (kk & 3) * 32;
+                            umma_ss(tmem + C::COL_S(b), sdesc_sw128(smem_u32(smem + C::OFF_K + oa), 16, 1024),
+                                    sdesc_sw128(smem_u32(sq + ob), 16, 1024), id_s, kk > 0);
+                        }
+#pragma unroll
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t oa = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
+                            const uint32_t ob = (kk >> 2) * 64 * 128 + (kk & 3) * 32;
+                            umma_ss(tmem + C::COL_DP(b), sdesc_sw128(smem_u32(smem + C::OFF_V + oa), 16, 1024),
+                                    sdesc_sw128(smem_u32(sdo + ob), 16, 1024), id_s, kk > 0);
+                        }
+                        umma_commit(s_full(b));
+                        // the previous item's products, while warpgroup b works on this one
+                        if (i > 0 && !post(prev_g, prev_st, i == 1)) { ok = false; break; }
+                        prev_g = gi;
+                        prev_st = st;
+                    }
+                    if (!ok) break;
+                    if (!post(prev_g, prev_st, items == 1)) break;
+                    umma_commit(dkv_full);
+                    umma_commit(kv_empty);
+                    ++unit_it;
+                }
+            }
+            __syncwarp();
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
+        // ------------------------------------------------------------ compute warpgroups (thread = key row)
+        const int gb = warp >> 2;                  // buffer / item parity of this warpgroup
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lb = tmem_lane_base(warp & 3);
+        const float c2 = p.scale_log2;
+        const float2 c2v = make_float2(c2, c2);
+        uint32_t unit_it = 0, q_it = 0, gi = 0;
+        bool ok = true;
+        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+            if (u >= p.num_units) continue;
+            const BUnit t = decode_bunit(p, u);
+            if (t.skip) continue;
+            const int kj = t.n0 + r;                 // key index inside the sequence
+            const bool kvalid = kj < t.Lk;
+            const size_t krow = (static_cast<size_t>(t.k_start) + kj) * p.Hkv + t.hk;
+            __nv_bfloat16* gdst = (gb == 0 ? p.dv : p.dk) + krow * D;
+            if (t.n_it == 0) {
+                if (kvalid) {
+                    const uint4 z = make_uint4(0, 0, 0, 0);
+                    for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(gdst)[c] = z;
+                }
+                continue;
+            }
+            // this key row is seen by query rows q_lo .. q_hi of the sequence (none if past the sequence)
+            int q_lo = -0x40000000, q_hi = 0x40000000;
+            if (p.wr >= 0) q_lo = kj - (t.Lk - t.Lq) - p.wr;
+            if (p.wl >= 0) q_hi = kj - (t.Lk - t.Lq) + p.wl;
+            if (!kvalid) q_lo = 0x40000000;
+            for (int it = 0; it < t.n_it && ok; ++it) {
+                for (int qh = 0; qh < 2; ++qh, ++q_it, ++gi) {
+                    if ((gi & 1) != static_cast<uint32_t>(gb)) continue;
+                    const int row0 = (t.m_start + it % t.n_m) * 128 + 64 * qh;
+                    const int st = q_it % ST;
+                    bool got = mbar_wait(s_full(gb), (gi >> 1) & 1, w);
+                    got = got && mbar_wait(q_full(st), (q_it / ST) & 1, w);
+                    if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                    tc_fence_after();
+                    // allowed item query columns: qmin .. qmax
+                    const int qmin = q_lo - row0, qmax = q_hi - row0;
+                    const bool any_mask = __any_sync(0xffffffffu, !(qmin <= 0 && qmax >= 63));
+                    const float* lse_t = sLSE + st * 64;
+                    const float* del_t = sDel + st * 64;
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        uint32_t sh[32], dh[32];
+                        tmem_ld32(tmem + lb + C::COL_S(gb) + 32 * half, sh);
+                        tmem_ld32(tmem + lb + C::COL_DP(gb) + 32 * half, dh);
+                        tmem_ld_wait_tie(sh);
+                        reg_tie(dh);
+                        uint32_t pp[16], dd[16];
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 l4 = *reinterpret_cast<const float4*>(lse_t + half * 32 + e);
+                            const float4 d4 = *reinterpret_cast<const float4*>(del_t + half * 32 + e);
+#pragma unroll
+                            for (int x = 0; x < 4; x += 2) {
+                                const float la = x == 0 ? l4.x : l4.z, lbv = x == 0 ? l4.y : l4.w;
+                                const float dla = x == 0 ? d4.x : d4.z, dlb = x == 0 ? d4.y : d4.w;
+                                const float2 sv = make_float2(__uint_as_float(sh[e + x]), __uint_as_float(sh[e + x + 1]));
+                                const float2 dv = make_float2(__uint_as_float(dh[e + x]), __uint_as_float(dh[e + x + 1]));
+                                const float2 a = ffma2(sv, c2v, make_float2(-la, -lbv));
+                                float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                                if (any_mask) {
+                                    const int qc = half * 32 + e + x;
+                                    pr.x = (qc >= qmin && qc <= qmax) ? pr.x : 0.f;
+                                    pr.y = (qc + 1 >= qmin && qc + 1 <= qmax) ? pr.y : 0.f;
+                                }
+                                const float2 ds = fmul2(pr, fadd2(dv, make_float2(-dla, -dlb)));
+                                pp[(e + x) / 2] = pack_bf16x2(pr.x, pr.y);
+                                dd[(e + x) / 2] = pack_bf16x2(ds.x, ds.y);
+                            }
+                        }
+                        // packed P^T, dS^T of item queries [32 half, +32) -> the 32 S^T columns just read
+                        tmem_st16(tmem + lb + C::COL_S(gb) + 32 * half, pp);
+                        tmem_st16(tmem + lb + C::COL_S(gb) + 32 * half + 16, dd);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(p_full(gb));
+                }
+            }
+            if (!ok) break;
+            // -------------------------------------------------- epilogue: warpgroup 0 writes dV, 1 writes dK
+            if (!mbar_wait(dkv_full, unit_it & 1, w)) { ok = false; break; }
+            ++unit_it;
+            tc_fence_after();
+            const uint32_t col = gb == 0 ? C::COL_DV : C::COL_DK;
+            const float mul = gb == 0 ? 1.f : p.scale;
+            const float2 mul2 = make_float2(mul, mul);
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t ra[32];
+                tmem_ld32(tmem + lb + col + cc * 32, ra);
+                tmem_ld_wait_tie(ra);
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float2 v = fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), mul2);
+                    pk[e] = pack_bf16x2(v.x, v.y);
+                }
+                if (kvalid) {
+                    uint4* o4 = reinterpret_cast<uint4*>(gdst + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(dkv_empty);
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) {
+        }
+    }
+    if (warp == MMA) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
 // ---------------------------------------------------------------------------- preprocess
 // One warp per (query token, head): Delta = sum_d dO * O (fp32), LSE2 = LSE * log2(e)
 // (+inf where LSE = -inf).  Also zeroes the dQ accumulator (grid-stride) unless dq_acc is NULL.
@@ -679,6 +1025,80 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
 }
 
+// Head dim 128, deterministic: the two-items-in-flight main kernel, then the dQ pass.
+static int run_bwd_pp(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
+                      void* dv, void* workspace, const Device& dev, cudaStream_t stream) {
+    using C = PPCfg;
+    constexpr int D = C::D;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    float* dq_acc = static_cast<float*>(workspace);
+    float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + up(static_cast<size_t>(pr.Tq) * pr.Hq * D * 4));
+    float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + up(static_cast<size_t>(pr.Tq) * pr.Hq * 4));
+    {
+        const long long rows = static_cast<long long>(pr.Tq) * pr.Hq;
+        long long blocks = (rows + 7) / 8;
+        const long long cap = static_cast<long long>(dev.num_sms) * 16;
+        if (blocks > cap) blocks = cap;
+        bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
+            static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
+            nullptr, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+        if (cudaPeekAtLastError() != cudaSuccess) return 5;
+    }
+    alignas(64) CUtensorMap mq, mk, mv, mdo;
+    const uint64_t rq = static_cast<uint64_t>(pr.Hq) * D * 2, rk = static_cast<uint64_t>(pr.Hkv) * D * 2;
+    if (!make_map_3d_bf16(&mq, pr.q, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, 64)) return 5;
+    if (!make_map_3d_bf16(&mdo, dout, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, 64)) return 5;
+    if (!make_map_3d_bf16(&mk, pr.k, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+    if (!make_map_3d_bf16(&mv, pr.v, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+
+    BwdParams p;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.dq_acc = dq_acc;
+    p.lse2 = lse2;
+    p.delta = delta;
+    p.cu_q = pr.cu_q;
+    p.cu_k = pr.cu_k;
+    p.num_seqs = pr.num_seqs;
+    p.Sq = pr.Sq;
+    p.Sk = pr.Sk;
+    p.Tq = pr.Tq;
+    p.Tk = pr.Tk;
+    p.Hq = pr.Hq;
+    p.Hkv = pr.Hkv;
+    p.group = pr.Hq / pr.Hkv;
+    p.n_blocks = (pr.Sk + 127) / 128;
+    const long long units = static_cast<long long>(p.n_blocks) * pr.num_seqs * pr.Hkv;
+    if (units > 0x7fffffffLL) return 2;
+    p.num_units = static_cast<int>(units);
+    p.scale = pr.scale;
+    p.scale_log2 = pr.scale * 1.4426950408889634f;
+    p.wl = pr.wl;
+    p.wr = pr.wr;
+    p.timeout_ns = dev.timeout_ns;
+    p.status = dev.status;
+
+    auto kern = bwd_pp_kernel;
+    static bool set[64] = {};
+    if (!set[dev.id & 63]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
+            cudaSuccess)
+            return 5;
+        // the setmaxnreg split assumes exactly LAUNCH_REGS per thread at launch
+        cudaFuncAttributes fa_attr;
+        if (cudaFuncGetAttributes(&fa_attr, kern) != cudaSuccess || fa_attr.numRegs != C::LAUNCH_REGS) return 2;
+        set[dev.id & 63] = true;
+    }
+    const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
+    if (grid > 0) {
+        prof_before(1, stream);
+        kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        prof_after(1, stream);
+        if (cudaPeekAtLastError() != cudaSuccess) return 5;
+    }
+    return launch_bwd_dq(pr, dout, lse2, delta, dq, dev, stream);
+}
+
 // Head dim 256: same preprocess, then the half-head-dim kernel of bwd256.cu (which also converts dQ).
 static int run_bwd256(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
                       void* dv, void* workspace, bool det, const Device& dev, cudaStream_t stream) {
@@ -707,7 +1127,7 @@ int launch_bwd(const Problem& pr, const void* out, const void* dout, const float
             return deterministic ? run_bwd<64, false>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream)
                                  : run_bwd<64, true>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
         case 128:
-            return deterministic ? run_bwd<128, false>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream)
+            return deterministic ? run_bwd_pp(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream)
                                  : run_bwd<128, true>(pr, out, dout, lse, dq, dk, dv, workspace, dev, stream);
         case 256: return run_bwd256(pr, out, dout, lse, dq, dk, dv, workspace, deterministic, dev, stream);
         default: return 2;
