@@ -119,7 +119,7 @@ struct BwdCfg {
     static constexpr uint32_t OFF_K = 0, OFF_V = T_BYTES, OFF_Q = 2 * T_BYTES, OFF_DO = (2 + ST) * T_BYTES,
                               OFF_DS = (2 + 2 * ST) * T_BYTES, OFF_STAT = OFF_DS + DS_BYTES,
                               OFF_BAR = OFF_STAT + 2 * ST * 128 * 4;
-    static constexpr int NUM_BARS = 2 + 2 * ST + 7;
+    static constexpr int NUM_BARS = 2 + 2 * ST + 9;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
     // tensor memory: dV | dK | S^T | dP^T.  After the gradient step the packed bf16 P^T and dS^T of each
     // 32-query half sit in that half's own 32 columns of S^T; dQ (fp32, D columns) is accumulated over
@@ -154,12 +154,15 @@ __global__ void __launch_bounds__(512, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     const uint32_t b0 = smem_u32(bars);
-    const uint32_t kv_full = b0, kv_empty = b0 + 8;
+    // K and V of a unit arrive / are released separately: V is last read by the unit's last dP^T,
+    // K by its last dQ (or S^T), so the next unit's V and first Q/dO tile load while those finish
+    const uint32_t k_full = b0, k_free = b0 + 8;
     auto q_full = [&](int s) { return b0 + 8u * (2 + s); };
     auto q_empty = [&](int s) { return b0 + 8u * (2 + ST + s); };
     // p_full / p_full_hi: compute warpgroup 0 (query columns 0-63) / 1 (64-127) done
     const uint32_t s_full = b0 + 8u * (2 + 2 * ST), p_full = s_full + 8, dq_full = s_full + 16,
-                   dq_empty = s_full + 24, dkv_full = s_full + 32, dq_empty_hi = s_full + 40, p_full_hi = s_full + 48;
+                   dq_empty = s_full + 24, dkv_full = s_full + 32, dq_empty_hi = s_full + 40, p_full_hi = s_full + 48,
+                   v_full = s_full + 56, v_free = s_full + 64;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PRODUCER = 12, MMA = 13;
@@ -182,6 +185,8 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bars + 2 + 2 * ST + 4, 1);    // dkv_full
         mbar_init(bars + 2 + 2 * ST + 5, 128);  // dq_empty_hi: dQ columns in the dP^T region read out
         mbar_init(bars + 2 + 2 * ST + 6, 128);  // p_full_hi: compute warpgroup 1 (query columns 64-127)
+        mbar_init(bars + 2 + 2 * ST + 7, 1);    // v_full
+        mbar_init(bars + 2 + 2 * ST + 8, 1);    // v_free
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -212,24 +217,13 @@ __global__ void __launch_bounds__(512, 1)
                 if (u >= p.num_units) continue;
                 const BUnit t = decode_bunit(p, u);
                 if (t.skip || t.n_it == 0) continue;
-                if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(kv_full, 2 * C::T_BYTES);
-#pragma unroll
-                    for (int c = 0; c < C::NCHUNK; ++c) {
-                        tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
-                                    t.k_start + t.n0);
-                        tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
-                                    t.k_start + t.n0);
-                    }
-                }
-                ++unit_it;
-                for (int it = 0; it < t.n_it; ++it, ++q_it) {
+                // one query tile's Q and dO (TMA) and statistics (plain loads) into the next ring stage
+                auto load_tile = [&](int it) -> bool {
                     const int g = it / t.n_m;
                     const int m0 = (t.m_start + it % t.n_m) * 128;
                     const int h = t.hk * G + g;
                     const int st = q_it % ST;
-                    if (q_it >= ST && !mbar_wait(q_empty(st), ((q_it / ST) - 1) & 1, w)) { ok = false; break; }
+                    if (q_it >= ST && !mbar_wait(q_empty(st), ((q_it / ST) - 1) & 1, w)) return false;
                     // tile statistics; rows past the sequence get LSE2 = +inf (P = 0) and Delta = 0
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -251,7 +245,30 @@ __global__ void __launch_bounds__(512, 1)
                         }
                     }
                     mbar_arrive(q_full(st));
+                    ++q_it;
+                    return true;
+                };
+                // V (free once the previous unit's last dP^T has run), the first Q / dO tile, then K
+                if (unit_it > 0 && !mbar_wait(v_free, (unit_it - 1) & 1, w)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(v_full, C::T_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, v_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
                 }
+                if (!load_tile(0)) { ok = false; break; }
+                if (unit_it > 0 && !mbar_wait(k_free, (unit_it - 1) & 1, w)) { ok = false; break; }
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(k_full, C::T_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, k_full, c * 64, t.hk,
+                                    t.k_start + t.n0);
+                }
+                ++unit_it;
+                for (int it = 1; it < t.n_it && ok; ++it)
+                    if (!load_tile(it)) ok = false;
             }
             __syncwarp();
         } else if (warp == MMA) {
@@ -266,8 +283,10 @@ __global__ void __launch_bounds__(512, 1)
                     if (u >= p.num_units) continue;
                     const BUnit t = decode_bunit(p, u);
                     if (t.skip || t.n_it == 0) continue;
-                    if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
+                    if (!mbar_wait(k_full, unit_it & 1, w)) { ok = false; break; }
+                    if (!mbar_wait(v_full, unit_it & 1, w)) { ok = false; break; }
                     for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
+                        const bool last = it + 1 == t.n_it;
                         const int st = q_it % ST;
                         if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
                         tc_fence_after();
@@ -279,6 +298,7 @@ __global__ void __launch_bounds__(512, 1)
                             umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + o), 16, 1024),
                                     sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
                         }
+                        if (!DQ && last) umma_commit(k_free);     // K's last reader without the dQ product
                         // dP^T goes where the previous tile's dQ was: both halves of it must be read out
                         if (DQ && g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
                         if (DQ && g_it > 0 && !mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
@@ -290,6 +310,7 @@ __global__ void __launch_bounds__(512, 1)
                                     sdesc_sw128(smem_u32(sdo + o), 16, 1024), id_kk, kk > 0);
                         }
                         umma_commit(s_full);
+                        if (last) umma_commit(v_free);            // V's last reader in this unit
                         // dV += P^T dO, dK += dS^T Q over queries 0-63, as soon as warpgroup 0 is done
                         if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
@@ -313,6 +334,7 @@ __global__ void __launch_bounds__(512, 1)
                                         id_dq, kk > 0);
                             }
                             umma_commit(dq_full);
+                            if (last) umma_commit(k_free);        // K's last reader in this unit
                         }
                         // dV, dK over queries 64-127
 #pragma unroll
@@ -326,7 +348,6 @@ __global__ void __launch_bounds__(512, 1)
                     }
                     if (!ok) break;
                     umma_commit(dkv_full);
-                    umma_commit(kv_empty);
                     ++unit_it;
                 }
             }
