@@ -411,11 +411,15 @@ __global__ void __launch_bounds__(512, 1)
             if (t.skip) continue;
             const int kj = t.n0 + r;                 // key index inside the sequence
             const bool kvalid = kj < t.Lk;
-            const size_t krow = (static_cast<size_t>(t.k_start) + kj) * p.Hkv + t.hk;
-            __nv_bfloat16* gdst = (gq == 0 ? p.dv : p.dk) + krow * D;
+            // this warpgroup's output row (dV for warpgroup 0, dK for 1)
+            auto out_row = [&](const BUnit& tt) {
+                const size_t krow = (static_cast<size_t>(tt.k_start) + tt.n0 + r) * p.Hkv + tt.hk;
+                return (gq == 0 ? p.dv : p.dk) + krow * D;
+            };
             if (t.n_it == 0) {
                 if (kvalid) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
+                    __nv_bfloat16* gdst = out_row(t);
                     for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(gdst)[c] = z;
                 }
                 continue;
@@ -497,22 +501,29 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t col = gq == 0 ? C::COL_DV : C::COL_DK;
             const float mul = gq == 0 ? 1.f : p.scale;
             const float2 mul2 = make_float2(mul, mul);
+            // rows go out through this warpgroup's half of the dS buffer: the last dQ product that read
+            // it is complete (dkv_full), and this warpgroup is its next writer
+            uint8_t* stg = smem + C::OFF_DS + gq * (C::DS_BYTES / 2) + (warp & 3) * 2048;
+            const BUnit te = decode_bunit(p, u);     // decoded again: nothing of it stays live over the tiles
+            __nv_bfloat16* gdst = out_row(te);
+            const int nvalid = min(max(te.Lk - te.n0 - (warp & 3) * 32, 0), 32);
+            const long long rstride = static_cast<long long>(p.Hkv) * D * 2;
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t ra[32];
                 tmem_ld32(tmem + lb + col + cc * 32, ra);
                 tmem_ld_wait_tie(ra);
-                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float2 v = fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), mul2);
-                    pk[e] = pack_bf16x2(v.x, v.y);
-                }
-                if (kvalid) {
-                    uint4* o4 = reinterpret_cast<uint4*>(gdst + cc * 32);
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v = fmul2(make_float2(__uint_as_float(ra[8 * q + 2 * e]), __uint_as_float(ra[8 * q + 2 * e + 1])), mul2);
+                        pk[e] = pack_bf16x2(v.x, v.y);
+                    }
+                    stg_put(stg, q, pk[0], pk[1], pk[2], pk[3]);
                 }
+                stg_flush(stg, reinterpret_cast<uint8_t*>(gdst + cc * 32), rstride, nvalid);
             }
             tc_fence_before();
         }

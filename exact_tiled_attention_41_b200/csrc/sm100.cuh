@@ -316,6 +316,31 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Row stores through shared memory: each lane puts the four 16-byte pieces of 64 bytes of its own row
+// into 2 KB of shared memory (stg, this warp's alone, 16-byte aligned; stg_put), then stg_flush writes
+// them so that each store instruction covers 8 rows x 64 contiguous bytes rather than 32 rows x 16
+// bytes: four times fewer cache lines per instruction.  Piece q of row r sits at 16-byte slot
+// 32 q + (r ^ q), so the row-wise writes and the piece-wise reads of every 8 lanes touch 8 different banks.
+__device__ __forceinline__ void stg_put(uint8_t* stg, int q, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+    const int lane = threadIdx.x & 31;
+    *reinterpret_cast<uint4*>(stg + ((q * 32 + (lane ^ q)) << 4)) = make_uint4(w0, w1, w2, w3);
+}
+
+// dst: this lane's destination of the 64 bytes (16-byte aligned); rows are row_stride bytes apart;
+// only the rows of lanes 0 .. nvalid-1 are written.  The warp may refill stg after this returns.
+__device__ __forceinline__ void stg_flush(const uint8_t* stg, uint8_t* dst, long long row_stride, int nvalid) {
+    const int lane = threadIdx.x & 31;
+    __syncwarp();
+    const int g = lane >> 2, c = lane & 3;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int rr = 4 * g + j;   // lanes 4g .. 4g+3 write row rr, 16 bytes each
+        const uint4 v = *reinterpret_cast<const uint4*>(stg + ((c * 32 + (rr ^ c)) << 4));
+        if (rr < nvalid) *reinterpret_cast<uint4*>(dst + (rr - lane) * row_stride + c * 16) = v;
+    }
+    __syncwarp();
+}
+
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 // Persistent schedule over work units sorted heaviest first: round k of CTA c takes unit
