@@ -560,7 +560,8 @@ struct PPCfg {
     static constexpr uint32_t KV_BYTES = 128 * D * 2;            // K or V tile: two [128 x 64] boxes
     static constexpr uint32_t IT_BYTES = 64 * D * 2;             // Q or dO item: two [64 x 64] boxes
     static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_Q = 2 * KV_BYTES, OFF_DO = OFF_Q + ST * IT_BYTES,
-                              OFF_STAT = OFF_DO + ST * IT_BYTES, OFF_BAR = OFF_STAT + 2 * ST * 64 * 4;
+                              OFF_STAT = OFF_DO + ST * IT_BYTES, OFF_STG = OFF_STAT + 2 * ST * 64 * 4,
+                              OFF_BAR = OFF_STG + 8 * 2048;   // 2 KB per compute warp for the output rows
     // kv_full, kv_empty, q_full[ST], q_empty[ST], s_full[2], p_full[2], dkv_full, dkv_empty
     static constexpr int NUM_BARS = 2 + 2 * ST + 4 + 2;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
@@ -853,22 +854,25 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t col = gb == 0 ? C::COL_DV : C::COL_DK;
             const float mul = gb == 0 ? 1.f : p.scale;
             const float2 mul2 = make_float2(mul, mul);
+            uint8_t* stg = smem + C::OFF_STG + warp * 2048;
+            const int nvalid = min(max(t.Lk - t.n0 - (warp & 3) * 32, 0), 32);
+            const long long rstride = static_cast<long long>(p.Hkv) * D * 2;
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t ra[32];
                 tmem_ld32(tmem + lb + col + cc * 32, ra);
                 tmem_ld_wait_tie(ra);
-                uint32_t pk[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float2 v = fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), mul2);
-                    pk[e] = pack_bf16x2(v.x, v.y);
-                }
-                if (kvalid) {
-                    uint4* o4 = reinterpret_cast<uint4*>(gdst + cc * 32);
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 v = fmul2(make_float2(__uint_as_float(ra[8 * q + 2 * e]), __uint_as_float(ra[8 * q + 2 * e + 1])), mul2);
+                        pk[e] = pack_bf16x2(v.x, v.y);
+                    }
+                    stg_put(stg, q, pk[0], pk[1], pk[2], pk[3]);
                 }
+                stg_flush(stg, reinterpret_cast<uint8_t*>(gdst + cc * 32), rstride, nvalid);
             }
             tc_fence_before();
             mbar_arrive(dkv_empty);

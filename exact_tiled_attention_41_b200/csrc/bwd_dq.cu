@@ -103,7 +103,10 @@ struct DqCfg {
     // s_full[2], dp_full, dp_free, ds_full[2], dq_full, dq_empty
     static constexpr int B1 = 2 + 2 * KST + 2 * VST;
     static constexpr int NUM_BARS = B1 + 8;
-    static constexpr size_t SMEM = 1024 + 2 * T_BYTES + (KST + VST) * KV_BYTES + NUM_BARS * 8 + 16;
+    // 2 KB per compute warp to write the dQ rows 8 at a time, where shared memory has room for it
+    static constexpr bool STAGE = 1024 + 2 * T_BYTES + (KST + VST) * KV_BYTES + 8 * 2048 + NUM_BARS * 8 + 16 <= 232448;
+    static constexpr uint32_t STG_BYTES = STAGE ? 8 * 2048 : 0;
+    static constexpr size_t SMEM = 1024 + 2 * T_BYTES + (KST + VST) * KV_BYTES + STG_BYTES + NUM_BARS * 8 + 16;
     static_assert(KST >= 2 && VST >= 1, "K_j is read by dQ_j after S_{j+1} is issued");
     static constexpr int THREADS = 384;
     static constexpr uint32_t S_COL(int s) { return s * BK; }
@@ -128,7 +131,8 @@ __global__ void __launch_bounds__(384, 1)
     uint8_t* sDO = sQ + C::T_BYTES;
     uint8_t* sK = sDO + C::T_BYTES;
     uint8_t* sV = sK + KST * C::KV_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VST * C::KV_BYTES);
+    uint8_t* sStg = sV + VST * C::KV_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + C::STG_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -374,16 +378,32 @@ __global__ void __launch_bounds__(384, 1)
                 uint32_t ra[32];
                 tmem_ld32(tmem + lb + C::DQ_COL + gw * (D / 2) + cc * 32, ra);
                 tmem_ld_wait_tie(ra);
-                uint32_t pk[16];
+                if constexpr (C::STAGE) {
+                    uint8_t* stg = sStg + warp * 2048;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const float2 v = fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), sc);
-                    pk[e] = pack_bf16x2(v.x, v.y);
-                }
-                if (valid) {
-                    uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t pk[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 v = fmul2(make_float2(__uint_as_float(ra[8 * q + 2 * e]), __uint_as_float(ra[8 * q + 2 * e + 1])), sc);
+                            pk[e] = pack_bf16x2(v.x, v.y);
+                        }
+                        stg_put(stg, q, pk[0], pk[1], pk[2], pk[3]);
+                    }
+                    stg_flush(stg, reinterpret_cast<uint8_t*>(dst + cc * 32), static_cast<long long>(p.Hq) * D * 2,
+                              min(max(t.Lq - (t.q0 + wq * 32), 0), 32));
+                } else {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float2 v = fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), sc);
+                        pk[e] = pack_bf16x2(v.x, v.y);
+                    }
+                    if (valid) {
+                        uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                    }
                 }
             }
             tc_fence_before();
