@@ -517,6 +517,52 @@ def measure_extras(torch, abi, A, W, dev, pk):
     return res
 
 
+def run_profile_case(args):
+    """One mid-size case of a single path, for an ncu capture: inputs larger than L2 but under a GB."""
+    import torch
+    from exact_tiled_attention_41_b200 import abi
+    from exact_tiled_attention_41_b200 import workloads as W
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    if args.profile_case == "decode":
+        # B=64, Hq=32, Hkv=8, D=128, cache lengths uniform in [1024, 2048], capacity 2048 (537 MB of cache)
+        B, Hq, Hkv, D, cap = 64, 32, 8, 128, 2048
+        w = W.kvcache(B, Hq, Hkv, D, cap, 1024, 2048, seed=0, nan_guard=False, device=str(dev))
+        t = w.tensors
+        lens = t["cache_seqlens"].to(dev)
+        out = torch.empty_like(t["q"])
+        lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=dev)
+        nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, 1, cap, D, 0)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        nbytes = float(t["cache_seqlens"].sum().item()) * Hkv * D * 2 * 2 + 2 * t["q"].numel() * 2
+        fn = lambda: abi.fa_fwd_kvcache(t["q"], t["k_cache"], t["v_cache"], lens, out, lse, B, Hq, Hkv, 1, cap, D,
+                                        w.scale, 0, 0, ws, nb, stream)
+        name = "decode_B64_Hq32_Hkv8_cap2048_D128"
+    else:
+        C, B, S, H, D = 4, 2, 8192, 32, 128
+        g = torch.Generator(str(dev)).manual_seed(3)
+        o_parts = torch.randn((C, B, S, H, D), generator=g, device=dev).to(torch.bfloat16)
+        l_parts = torch.randn((C, B, H, S), generator=g, device=dev)
+        o_m = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
+        l_m = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+        nbytes = (C + 1) * (o_m.numel() * 2 + l_m.numel() * 4)
+        fn = lambda: abi.fa_merge_lse(o_parts, l_parts, C, B, S, H, D, 0, o_m, l_m, 0, stream)
+        name = "merge_lse_4parts_B2_S8192_H32_D128"
+    for _ in range(args.warmup):
+        if fn() != 0:
+            raise RuntimeError(f"{name}: the call failed")
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / max(args.steps, 1)
+    print(json.dumps({"profile_case": name, "ms": ms, "gbs": nbytes / ms / 1e6, "algorithmic_bytes": nbytes}))
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -528,12 +574,16 @@ def main():
                     help="time the step with the deterministic backward (dq from the query-tile-stationary pass)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--profile-case", choices=["decode", "merge"], default=None,
+                    help="run only a mid-size case of one path (inputs > L2, < 1 GB), e.g. under ncu, and print its time")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.profile_case is not None:
+        return run_profile_case(args)
     if args.impl == "reference":
         return run_reference(args, rank, world)
     import torch
