@@ -420,7 +420,7 @@ def measure_extras(torch, abi, A, W, dev, pk):
         "bwd_frac_of_measured_peak": 2.5 * wf / wbms / 1e9 / pk["bf16_tflops"]}
     del t, out, lse, dq, dk, dv, ws
 
-    # varlen packed batch, D = 64 and 256 (forward; backward for D = 64)
+    # varlen packed batch, D = 64 and 256 (forward and backward)
     for D in (64, 256):
         w = W.varlen_packed(D, seed=0)
         t = {n: x.to(dev) for n, x in w.tensors.items()}
@@ -433,14 +433,13 @@ def measure_extras(torch, abi, A, W, dev, pk):
                                               m["max_k"], m["total_q"], m["total_k"], 16, 16, D, w.scale, 1, None, 0,
                                               stream), 5)
         r = {"fwd_ms": fms, "fwd_tflops": ff / fms / 1e9, "total_tokens": m["total_q"]}
-        if D == 64:
-            dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
-            nb = abi.fa_varlen_bwd_workspace_size(16, m["total_q"], m["total_k"], 16, 16, D)
-            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
-            bms = timed(lambda: abi.fa_varlen_bwd(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, t["cu_q"],
-                                                  t["cu_k"], 16, m["max_q"], m["max_k"], m["total_q"], m["total_k"], 16,
-                                                  16, D, w.scale, 1, ws, nb, stream), 3)
-            r.update(bwd_ms=bms, bwd_tflops=2.5 * ff / bms / 1e9)
+        dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+        nb = abi.fa_varlen_bwd_workspace_size(16, m["total_q"], m["total_k"], 16, 16, D)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        bms = timed(lambda: abi.fa_varlen_bwd(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, t["cu_q"],
+                                              t["cu_k"], 16, m["max_q"], m["max_k"], m["total_q"], m["total_k"], 16,
+                                              16, D, w.scale, 1, ws, nb, stream), 3)
+        r.update(bwd_ms=bms, bwd_tflops=2.5 * ff / bms / 1e9)
         res[f"varlen_16seq_H16_D{D}_causal"] = r
         del t
 
