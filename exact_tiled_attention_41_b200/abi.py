@@ -39,6 +39,7 @@ FA_KERNEL_FWD = 0
 FA_KERNEL_BWD = 1
 FA_KERNEL_DECODE = 2
 FA_KERNEL_BWD_DQ = 3
+FA_KERNEL_BWD_ALL = 4
 
 _P = ctypes.c_void_p
 _I = ctypes.c_int

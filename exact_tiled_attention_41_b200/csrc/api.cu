@@ -81,6 +81,18 @@ int get_device(Device* d) {
 
 using namespace fa;
 
+namespace {
+// The whole backward of one call (preprocess, main kernel, dQ convert or dQ pass) between one pair
+// of profiling events (id FA_KERNEL_BWD_ALL).
+int launch_bwd_timed(const Problem& pr, const void* out, const void* dout, const float* lse, void* dq, void* dk,
+                     void* dv, void* workspace, bool deterministic, const Device& dev, cudaStream_t stream) {
+    prof_before(4, stream);
+    const int st = launch_bwd(pr, out, dout, lse, dq, dk, dv, workspace, deterministic, dev, stream);
+    prof_after(4, stream);
+    return st;
+}
+}  // namespace
+
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 static bool supported_d(int D) { return D == 64 || D == 128 || D == 256; }
@@ -234,8 +246,8 @@ int fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, cons
     Device dev;
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
     Problem pr = dense_problem(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, window_left, window_right);
-    return launch_bwd(pr, out, dout, lse, dq, dk, dv, workspace, deterministic != 0, dev,
-                      static_cast<cudaStream_t>(stream));
+    return launch_bwd_timed(pr, out, dout, lse, dq, dk, dv, workspace, deterministic != 0, dev,
+                            static_cast<cudaStream_t>(stream));
 }
 
 // ----------------------------------------------------------------------- varlen
@@ -342,8 +354,8 @@ int fa_varlen_bwd_ex(const void* q, const void* k, const void* v, const void* ou
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
     Problem pr = varlen_problem(q, k, v, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
                                 total_k, Hq, Hkv, D, softmax_scale, causal, window_left, window_right);
-    return launch_bwd(pr, out, dout, lse, dq, dk, dv, workspace, deterministic != 0, dev,
-                      static_cast<cudaStream_t>(stream));
+    return launch_bwd_timed(pr, out, dout, lse, dq, dk, dv, workspace, deterministic != 0, dev,
+                            static_cast<cudaStream_t>(stream));
 }
 
 // ----------------------------------------------------------------------- KV-cache decode

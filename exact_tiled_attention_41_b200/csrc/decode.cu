@@ -105,8 +105,14 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
     return static_cast<uint32_t>(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Two CTAs per SM up to D = 128 (3 stages of 2 x 64 keys x D); at D = 256 a stage is 64 KB and the
+// output fragments alone take 128 registers per thread, so one CTA per SM (the 3-stage ring still
+// keeps 128 KB of K/V in flight per SM).
 template <int D>
-__global__ void __launch_bounds__((kDecConsumers + 1) * 32, 2)
+constexpr int dec_min_blocks() { return D == 256 ? 1 : 2; }
+
+template <int D>
+__global__ void __launch_bounds__((kDecConsumers + 1) * 32, dec_min_blocks<D>())
     decode_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ DecodeParams p) {
     constexpr int NBOX = D / 64;
@@ -461,7 +467,7 @@ int kvcache_validate(const KvCall& c, bool pointers) {
         return FA_ERR_INVALID_ARG;
     if (c.Hq <= 0 || c.Hkv <= 0 || c.Hq % c.Hkv != 0) return FA_ERR_INVALID_ARG;
     if (!(c.scale > 0.f) || !isfinite(c.scale)) return FA_ERR_INVALID_ARG;
-    if (c.D != 64 && c.D != 128) return FA_ERR_UNSUPPORTED;
+    if (c.D != 64 && c.D != 128 && c.D != 256) return FA_ERR_UNSUPPORTED;
     if (pointers) {
         if ((c.k_new == nullptr) != (c.v_new == nullptr)) return FA_ERR_INVALID_ARG;
         if ((c.seqlen_new > 0) != (c.k_new != nullptr)) return FA_ERR_INVALID_ARG;
@@ -591,6 +597,7 @@ int kvcache_launch(const KvCall& c, int chunk, void* workspace, const Device& de
     switch (c.D) {
         case 64: return run_decode<64>(c, chunk, workspace, dev, stream);
         case 128: return run_decode<128>(c, chunk, workspace, dev, stream);
+        case 256: return run_decode<256>(c, chunk, workspace, dev, stream);
         default: return FA_ERR_UNSUPPORTED;
     }
 }

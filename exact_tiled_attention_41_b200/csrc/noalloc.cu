@@ -1,9 +1,9 @@
 // noalloc.cu -- fa_fwd_kvcache_noalloc: KV-cache decode that needs no caller workspace.
 //
 // Some callers cannot allocate device memory at the point where they decode:
-// code running inside a CUDA-graph capture that must not grow the pool, plugins
-// and inference runtimes that hand a kernel only the tensors they own, or C
-// programs with no allocator of their own.  This entry point runs the same
+// plugins and inference runtimes that plan all device memory ahead of time and
+// hand a kernel only the tensors they own, or C programs with no allocator of
+// their own, so a per-call workspace has nowhere to come from.  This entry point runs the same
 // split-KV decode as fa_fwd_kvcache, but keeps the per-split partial outputs
 // and log-sum-exps in a fixed array compiled into the library.
 //
@@ -23,8 +23,9 @@ constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-// Device address of g_noalloc_scratch per device.  The host-side symbol is only
-// a stand-in for the device array and must never be handed to a kernel.
+// Device address of g_noalloc_scratch per device, looked up by the first call on that device
+// and kept for the life of the process (a cudaDeviceReset after that is not supported).  The
+// host-side symbol is only a stand-in for the device array and must never be handed to a kernel.
 void* g_scratch_ptr[64] = {};
 
 int scratch_for_current_device(const Device& dev, void** out) {

@@ -7,7 +7,7 @@
 namespace fa {
 
 namespace {
-constexpr int kIds = 4;
+constexpr int kIds = 5;
 constexpr int kMaxRec = 1024;
 struct Rec {
     cudaEvent_t start[kMaxRec];

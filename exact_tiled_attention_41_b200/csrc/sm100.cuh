@@ -110,6 +110,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Bring a 3-D tile into L2 ahead of its load (no shared-memory destination, no completion signal).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap* map, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 // Make generic-proxy writes to shared memory visible to the async proxy (tensor cores, TMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -287,28 +295,38 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
     return r;
 }
 
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    uint64_t d, x, y;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "f"(b.x), "f"(b.y));
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(x), "l"(y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+
 // Two exp2 on the FMA pipe, for the share of the softmax exponentials taken off the
-// multi-function unit.  x = j + f with j = rint(x) (rounding by adding and subtracting
-// 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f is a degree-6 polynomial whose coefficients minimise the
-// maximum relative error on [-1/2, 1/2] (Remez exchange, csrc/fit_exp2_poly.py): worst relative
-// error 1.0e-7 in fp32 over [-126, 8], about 2 ulp, like the hardware ex2.approx.  2^j is applied
-// by adding j to the exponent field (the shift drops the bias bits of the rounding constant).
-// Arguments below -125 (including -inf) give exactly 0 (results under 2^-125 are dropped, as
-// ex2.approx.ftz drops those under 2^-126; the exponent add stays in the normal range); x <= 127.
+// multi-function unit.  x is clamped to >= -126, then split as x = j + f with j = rint(x)
+// (adding 1.5 * 2^23 leaves rint(x) in the low mantissa bits of t) and f in [-1/2, 1/2];
+// 2^f is the degree-5 polynomial whose coefficients minimise the maximum relative error on
+// [-1/2, 1/2] (Remez exchange; exact_tiled_attention_41_b200/fit_exp2_poly.py prints them), and
+// 2^j is applied by adding j to the exponent field (t << 23 keeps only j's bits there).  Worst
+// relative error 2.3e-7 over [-125, 8] (about 2 ulp, the class of the hardware ex2.approx).
+// Below -125 the result is a non-negative value under 2^-125 rather than exactly 0, so the
+// softmax calls this only on tiles without masked (-inf) scores; x <= 127.
 __device__ __forceinline__ float2 exp2_fma2(float2 x) {
     constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    const float2 t = fadd2(x, make_float2(kRound, kRound));
-    const float2 nj = fadd2(make_float2(kRound, kRound), make_float2(-t.x, -t.y));   // -rint(x)
-    const float2 f = fadd2(x, nj);
-    float2 p = ffma2(make_float2(1.5345812e-4f, 1.5345812e-4f), f, make_float2(1.3399931e-3f, 1.3399931e-3f));
-    p = ffma2(p, f, make_float2(9.618489e-3f, 9.618489e-3f));
-    p = ffma2(p, f, make_float2(5.5503286e-2f, 5.5503286e-2f));
-    p = ffma2(p, f, make_float2(2.4022646e-1f, 2.4022646e-1f));
-    p = ffma2(p, f, make_float2(6.931472e-1f, 6.931472e-1f));
-    p = ffma2(p, f, make_float2(1.0f, 1.0f));
+    const float2 xc = make_float2(fmaxf(x.x, -126.f), fmaxf(x.y, -126.f));
+    const float2 t = fadd2(xc, make_float2(kRound, kRound));
+    const float2 f = fsub2(xc, fsub2(t, make_float2(kRound, kRound)));   // x - rint(x)
+    float2 p = ffma2(make_float2(1.3276472e-3f, 1.3276472e-3f), f, make_float2(9.675541e-3f, 9.675541e-3f));
+    p = ffma2(p, f, make_float2(5.550713e-2f, 5.550713e-2f));
+    p = ffma2(p, f, make_float2(2.402212e-1f, 2.402212e-1f));
+    p = ffma2(p, f, make_float2(6.9314694e-1f, 6.9314694e-1f));
+    p = ffma2(p, f, make_float2(1.0000001f, 1.0000001f));
     const uint32_t bx = __float_as_uint(p.x) + (__float_as_uint(t.x) << 23);
     const uint32_t by = __float_as_uint(p.y) + (__float_as_uint(t.y) << 23);
-    return make_float2(x.x < -125.f ? 0.f : __uint_as_float(bx), x.y < -125.f ? 0.f : __uint_as_float(by));
+    return make_float2(__uint_as_float(bx), __uint_as_float(by));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

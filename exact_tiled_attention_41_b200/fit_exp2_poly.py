@@ -1,6 +1,6 @@
 """Fit the polynomial used for the FMA-pipe half of exp2 in the softmax kernels.
 
-    python exact_tiled_attention_41_b200/csrc/fit_exp2_poly.py
+    python -m exact_tiled_attention_41_b200.fit_exp2_poly
 
 2^x is split as 2^j * 2^f with j = round(x) and f = x - j in [-1/2, 1/2]; 2^f is
 approximated by a degree-5 polynomial p(f) whose maximum *relative* error on
@@ -8,6 +8,8 @@ approximated by a degree-5 polynomial p(f) whose maximum *relative* error on
 the weighted error p(f)/2^f - 1 at 7 points).  The script prints the
 coefficients (highest degree first, as used by Horner's rule in sm100.cuh) and
 the worst relative error of the fp32 Horner evaluation against float64 2^x.
+exp2_fma2 in csrc/sm100.cuh uses exactly the printed float32 values (a CPU test
+re-runs the fit and compares them with the header).
 """
 
 import numpy as np
@@ -58,7 +60,7 @@ def remez(deg=DEG, iters=30):
 
 def fp32_horner_error(c):
     c32 = np.asarray(c[::-1], dtype=np.float32)      # highest degree first
-    x = np.linspace(-126.0, 8.0, 4_000_001).astype(np.float32)
+    x = np.linspace(-125.0, 8.0, 4_000_001).astype(np.float32)
     j = np.rint(x).astype(np.float32)
     f = (x - j).astype(np.float32)
     p = np.full_like(f, c32[0])
@@ -69,8 +71,13 @@ def fp32_horner_error(c):
     return np.max(np.abs(y / ref - 1.0))
 
 
+def coefficients_f32(deg=DEG):
+    """The fitted coefficients rounded to float32, highest degree first."""
+    return [np.float32(a) for a in remez(deg)[::-1]]
+
+
 if __name__ == "__main__":
     c = remez()
     for i, a in enumerate(c[::-1]):
         print(f"c{DEG - i} = {np.float32(a)!r}  ({a:.17g})")
-    print("max relative error (fp32 Horner) over [-126, 8]:", fp32_horner_error(c))
+    print("max relative error (fp32 Horner) over [-125, 8]:", fp32_horner_error(c))

@@ -190,7 +190,9 @@ FA_API int fa_varlen_bwd_ex(const void* q, const void* k, const void* v, const v
  * automatically; > 0 asks for that many splits of cache_capacity.  The result
  * does not depend on the split except through float32 rounding.
  * Workspace (fa_fwd_kvcache_workspace_size): float32 partial outputs and LSEs.
- * Head dims 64 and 128.  No backward (the docstring states the same).
+ * Head dims 64, 128 and 256.  No backward (the docstring states the same).
+ * The automatic split (num_splits = 0) is sized for 148 SMs (B200) whatever
+ * the device, so the workspace size does not depend on the device it runs on.
  */
 FA_API size_t fa_fwd_kvcache_workspace_size(int B, int Hq, int Hkv, int Sq, int cache_capacity, int D, int num_splits);
 FA_API int fa_fwd_kvcache(const void* q, const void* k_cache, const void* v_cache, const int32_t* cache_seqlens,
@@ -259,9 +261,9 @@ FA_API int fa_merge_lse(const void* o_parts, const float* lse_parts, int num_par
 
 /* ------------------------------------------------------------------------- KV-cache decode without caller memory
  * fa_fwd_kvcache_noalloc: the same computation as fa_fwd_kvcache, for callers
- * that cannot allocate device memory when they decode -- for example code that
- * runs while a CUDA graph is being captured and must not grow a memory pool,
- * or a plugin / runtime that only receives the tensors it owns.  The source
+ * that cannot allocate device memory when they decode -- for example a plugin or
+ * inference runtime that plans its device memory ahead of time and only receives
+ * the tensors it owns, or a C program with no allocator of its own.  The source
  * pages have no counterpart of this entry point; it is an interface addition.
  *
  * The per-split partial results live in one array compiled into the library
@@ -271,11 +273,14 @@ FA_API int fa_merge_lse(const void* o_parts, const float* lse_parts, int num_par
  * fa_fwd_kvcache; no workspace argument, and nothing is allocated or freed.
  *   - The first call on a device looks up the array's device address there
  *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     The address is kept for the life of the process: calling it again after a
+ *     cudaDeviceReset of that device is not supported.
  *   - All calls share the array: calls that overlap on the GPU (other streams,
  *     other host threads) race on it and must be serialised by the caller.
  *     Nothing in it needs to start at zero; each call writes what it reads.
  *   - With num_splits = 0 the split is chosen as for fa_fwd_kvcache and made
- *     coarser until the partials fit.  If they cannot fit (an explicit
+ *     coarser (doubled, at most to the whole capacity) until the partials fit;
+ *     when no coarsening is needed the result is bit-identical to fa_fwd_kvcache's.  If they cannot fit (an explicit
  *     num_splits too large, or B * Sq * Hq * (D + 1) * 4 bytes beyond the array),
  *     the call returns FA_ERR_WORKSPACE and launches nothing.
  */
@@ -307,14 +312,18 @@ FA_API unsigned long long fa_set_wait_timeout_ns(unsigned long long ns);
  * every later launch of the main kernel of fa_fwd / fa_varlen_fwd (id 0), the
  * main backward kernel of fa_bwd / fa_varlen_bwd (id 1), the split kernel of
  * fa_fwd_kvcache (id 2) and the dQ pass of the deterministic backward (id 3)
- * record a pair of CUDA events around itself on the
+ * record a pair of CUDA events around itself, and every fa_bwd / fa_varlen_bwd
+ * call records one pair around all of its launches (id 4: preprocess, main
+ * kernel and dQ convert or dQ pass), on the
  * launching stream (up to 1024 launches per id; later ones are not recorded),
  * and clears earlier records; fa_profile_begin(0) stops recording.
  * fa_profile_read, after the caller has synchronised those streams, returns the
  * number of recorded launches of `kernel_id` and the sum of their durations in
  * milliseconds.  Events are created on first use; no device memory is allocated.
  */
-enum fa_kernel_id { FA_KERNEL_FWD = 0, FA_KERNEL_BWD = 1, FA_KERNEL_DECODE = 2, FA_KERNEL_BWD_DQ = 3 };
+enum fa_kernel_id {
+    FA_KERNEL_FWD = 0, FA_KERNEL_BWD = 1, FA_KERNEL_DECODE = 2, FA_KERNEL_BWD_DQ = 3, FA_KERNEL_BWD_ALL = 4
+};
 FA_API int fa_profile_begin(int enable);
 FA_API int fa_profile_read(int kernel_id, int* launches, float* total_ms);
 

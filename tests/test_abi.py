@@ -153,7 +153,7 @@ def _kv_ex(**kw):
     (dict(block_table=FAKE, max_blocks_per_seq=0, cache_capacity=256), abi.FA_ERR_INVALID_ARG),
     (dict(block_table=FAKE, max_blocks_per_seq=4, cache_capacity=256, cache_batch_idx=FAKE), abi.FA_ERR_INVALID_ARG),
     (dict(cache_batch=0), abi.FA_ERR_INVALID_ARG),
-    (dict(D=256), abi.FA_ERR_UNSUPPORTED),
+    (dict(D=512), abi.FA_ERR_UNSUPPORTED),
     (dict(workspace_bytes=0), abi.FA_ERR_WORKSPACE),
     (dict(block_table=FAKE + 2, max_blocks_per_seq=4, cache_capacity=256), abi.FA_ERR_ALIGNMENT),
 ])

@@ -39,7 +39,7 @@ def run_and_check(w, causal, window=(-1, -1), num_splits=0):
     return out, lse
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("Sq", [2, 5, 16])
 def test_multi_query_causal(D, Sq):
     lens = [Sq, 63, 64, 65, 700, 1023]
@@ -55,7 +55,7 @@ def test_append_then_attend(num_splits):
     run_and_check(w, True, num_splits=num_splits)
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 def test_paged_cache_with_append(D):
     lens = [0, 255, 256, 257, 900, 1400]
     w = W.kvcache_update(len(lens), 4, 8, 2, D, 1536, lens, seqlen_new=4, page=256, seed=50 + D)
@@ -99,3 +99,16 @@ def test_bad_block_id_is_reported_not_read():
     torch.cuda.synchronize()
     assert abi.fa_get_device_status() == abi.FA_ERR_INVALID_ARG
     assert abi.fa_get_device_status() == 0
+
+
+@pytest.mark.parametrize("num_splits", [0, 1, 3])
+def test_head_dim_256_single_token(num_splits):
+    # README: head dims up to 256; NaN guards in every cache row past the lengths
+    lens = [1, 63, 64, 65, 1000, 2047, 0]
+    w = W.kvcache_update(len(lens), 1, 16, 4, 256, 2048, lens, seed=100 + num_splits)
+    run_and_check(w, False, num_splits=num_splits)
+
+
+def test_head_dim_256_paged_single_token():
+    lens = [1, 511, 512, 1000]
+    run_and_check(W.kvcache_update(4, 1, 8, 2, 256, 1024, lens, page=256, seed=110), False)

@@ -1,0 +1,126 @@
+"""GPU parity on inputs built to drive the forward's exact O rescale.
+
+The forward keeps each row's exponentials, row sum and O accumulator against one reference
+max and moves that reference (rescaling O in tensor memory) only when a new tile's row max
+exceeds it by more than 8 in log2 units (FlashAttention fork v1.4 notes, section 4,
+softmax_rescale_o: every change of the max must rescale O; the exact variant required here
+never skips one).  On N(0, 1) inputs the first tile almost always holds a row's max, so the
+rescale branch is rarely taken.  Here keys carry a component along one direction whose size
+grows tile by tile, and queries carry that direction with a per-row weight, so the scores of a
+row rise (or fall) by a set amount from one 128-key tile to the next:
+
+  * rise > 8 log2 units per tile: the reference moves, and O is rescaled, at every tile;
+  * rise between 0 and 8 log2 units: the reference moves only every second or third tile, so
+    the deferred rows keep P, l and O on an older reference in between;
+  * rows with a negative weight see falling scores (no rescale after their first tile), mixed
+    with rising rows inside every warp.
+
+Each case is checked against the fp64 oracle (forward O, LSE, and the backward, which
+recomputes P from the LSE) at the stated tolerances, and a numpy model of the tiled loop
+with the O rescale left out shows that such a slip would miss those tolerances by far.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_tiled_attention_41_b200 import workloads as W
+from tests import gpu_helpers as H
+
+pytestmark = pytest.mark.gpu
+
+TILE = 128
+LOG2E = 1.4426950408889634
+
+
+def _rising(q, k, seg_starts, seg_lens, D, rise_log2, g):
+    """Add the ramp along coordinate 0: key j of a sequence gets a * (tile of j), query i gets b_i.
+
+    scale * b * a = rise_log2 / log2(e) natural units per tile for rows with b_i = b; b_i takes
+    the values b, -b, b/2 and 3b/4 in a seeded pattern (all exact in bf16)."""
+    scale = 1.0 / math.sqrt(D)
+    step_nat = rise_log2 / LOG2E
+    b = 4.0 if D <= 64 else 8.0
+    a = step_nat / (scale * b)            # per-tile step of the key component
+    weights = torch.tensor([b, -b, b / 2, 3 * b / 4])
+    for s0, n in zip(seg_starts, seg_lens):
+        tiles = torch.arange(n) // TILE
+        k[s0:s0 + n, :, 0] = (tiles.float() * a).to(torch.bfloat16)[:, None]
+        pick = torch.randint(0, 4, (n, q.shape[1]), generator=g)
+        q[s0:s0 + n, :, 0] = weights[pick].to(torch.bfloat16)
+    return q, k
+
+
+def _dense_case(D, causal, rise_log2, seed):
+    w = W.dense(1, 512, 512, 4, 2, D, causal, seed=seed)
+    g = torch.Generator("cpu").manual_seed(seed + 1000)
+    q = w.tensors["q"][0].clone()
+    k = w.tensors["k"][0].clone()
+    q, k = _rising(q, k, [0], [512], D, rise_log2, g)
+    w.tensors["q"], w.tensors["k"] = q[None], k[None]
+    return w
+
+
+def _varlen_case(D, causal, rise_log2, seed):
+    lens = [300, 517, 129]
+    w = W.varlen(lens, lens, 4, 2, D, causal, seed=seed)
+    g = torch.Generator("cpu").manual_seed(seed + 1000)
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).tolist()
+    w.tensors["q"], w.tensors["k"] = _rising(w.tensors["q"].clone(), w.tensors["k"].clone(), starts, lens, D,
+                                             rise_log2, g)
+    return w
+
+
+def _skip_rescale_model(qh, kh, vh, scale, causal):
+    """Tiled online softmax of one head (fp64) with the O rescale left out: O keeps the
+    contributions of earlier tiles at their old reference while l is rescaled."""
+    Sq, Sk = qh.shape[0], kh.shape[0]
+    s = scale * qh @ kh.T
+    if causal:
+        s = np.where(np.arange(Sk)[None, :] <= np.arange(Sq)[:, None] + (Sk - Sq), s, -np.inf)
+    m = np.full(Sq, -np.inf)
+    l = np.zeros(Sq)
+    o = np.zeros((Sq, vh.shape[1]))
+    for t0 in range(0, Sk, TILE):
+        st = s[:, t0:t0 + TILE]
+        m_new = np.maximum(m, st.max(axis=1))
+        ok = np.isfinite(m_new)
+        ref = np.where(ok, m_new, 0.0)
+        alpha = np.where(np.isfinite(m), np.exp(m - ref), 0.0)
+        p = np.exp(st - ref[:, None])
+        l = l * alpha + p.sum(axis=1)
+        o = o + p @ vh[t0:t0 + TILE]          # the slip: O is not multiplied by alpha
+        m = m_new
+    return o / np.where(l > 0, l, 1.0)[:, None]
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("rise_log2", [9.0, 3.0])
+def test_dense_rising_scores(D, causal, rise_log2):
+    w = _dense_case(D, causal, rise_log2, seed=D + 10 * causal + int(rise_log2))
+    H.check_dense(w)
+    if rise_log2 > 8.0:
+        # the inputs make the rescale matter: leaving it out would be far outside the tolerance
+        t = w.tensors
+        qh, kh, vh = H.f64(t["q"][0, :, 0]), H.f64(t["k"][0, :, 0]), H.f64(t["v"][0, :, 0])
+        o_ref, _ = oracle.mha_forward(H.f64(t["q"]), H.f64(t["k"]), H.f64(t["v"]), w.scale, causal)
+        bad = _skip_rescale_model(qh, kh, vh, w.scale, causal)
+        assert np.abs(bad - o_ref[0, :, 0]).max() > 10 * H.O_TOL
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("rise_log2", [9.0, 3.0])
+def test_varlen_rising_scores(D, causal, rise_log2):
+    w = _varlen_case(D, causal, rise_log2, seed=7 * D + causal + int(rise_log2))
+    H.check_varlen(w)
+
+
+@pytest.mark.parametrize("rise_log2", [9.0, 3.0])
+def test_rising_scores_deterministic_backward(rise_log2):
+    w = _dense_case(128, True, rise_log2, seed=77)
+    H.check_dense(w, deterministic=True)

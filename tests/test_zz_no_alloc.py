@@ -1,17 +1,22 @@
 """fa_fwd_kvcache_noalloc: KV-cache decode for callers that cannot allocate device
-memory when they decode (code inside a CUDA-graph capture that must not grow a
-memory pool, plugins or runtimes that only receive the tensors they own).  Its
+memory when they decode (plugins or runtimes that plan their device memory ahead of
+time and only receive the tensors they own, C programs without an allocator).  Its
 partial results live in a fixed array inside the library instead of a caller
-workspace; the results must match fa_fwd_kvcache's, here on two calls in a row
-with different inputs, so leftovers of the first call cannot leak into the second.
+workspace.  Where it uses the same split as fa_fwd_kvcache the results must be
+bit-identical to that entry point's, here on two calls in a row with different
+inputs, so leftovers of the first call cannot leak into the second; where the fixed
+array forces a coarser split the result must match fa_fwd_kvcache run with that
+split, and the fp64 oracle within the stated tolerances.
 
 This file is named to be collected last: a run that stops at the first failure
 has then already run every other test.
 """
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from exact_tiled_attention_41_b200 import abi, workloads as W
 from tests import gpu_helpers as H
 
@@ -20,13 +25,24 @@ pytestmark = pytest.mark.gpu
 FAKE = 0x10000
 
 
-def _reference(t, B, Hq, Hkv, cap, D, scale):
+def _reference(t, B, Hq, Hkv, cap, D, scale, num_splits=0):
     out = torch.empty_like(t["q"])
     lse = torch.empty((B, Hq, 1), dtype=torch.float32, device="cuda")
-    nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, 1, cap, D, 0)
+    nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, 1, cap, D, num_splits)
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
     assert abi.fa_fwd_kvcache(t["q"], t["k_cache"], t["v_cache"], t["cache_seqlens"], out, lse, B, Hq, Hkv, 1, cap,
-                              D, scale, 0, 0, ws, nb) == 0
+                              D, scale, 0, num_splits, ws, nb) == 0
+    return out, lse
+
+
+def _noalloc(t, B, Hq, Hkv, cap, D, scale):
+    out = torch.full_like(t["q"], float("nan"))
+    lse = torch.full((B, Hq, 1), float("nan"), dtype=torch.float32, device="cuda")
+    st = abi.fa_fwd_kvcache_noalloc(t["q"], t["k_cache"], t["v_cache"], t["cache_seqlens"], out, lse, B, Hq, Hkv,
+                                    1, cap, D, scale, 0, 0)
+    assert st == 0, abi.status_string(st)
+    torch.cuda.synchronize()
+    assert abi.fa_get_device_status() == 0
     return out, lse
 
 
@@ -37,15 +53,34 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(D):
         w = W.kvcache(B, Hq, Hkv, D, cap, 0, 0, seed=seed + D, lengths=lengths)
         t = {n: x.cuda() for n, x in w.tensors.items()}
         ref_out, ref_lse = _reference(t, B, Hq, Hkv, cap, D, w.scale)
-        out = torch.full_like(t["q"], float("nan"))
-        lse = torch.full((B, Hq, 1), float("nan"), dtype=torch.float32, device="cuda")
-        st = abi.fa_fwd_kvcache_noalloc(t["q"], t["k_cache"], t["v_cache"], t["cache_seqlens"], out, lse, B, Hq, Hkv,
-                                        1, cap, D, w.scale, 0, 0)
-        assert st == 0, abi.status_string(st)
-        torch.cuda.synchronize()
-        assert abi.fa_get_device_status() == 0
-        H.check_o(out, H.f64(ref_out))
-        H.check_lse(lse, H.f64(ref_lse))
+        out, lse = _noalloc(t, B, Hq, Hkv, cap, D, w.scale)
+        # same split, same kernels: the same bits (an empty row gives 0 / -inf in both)
+        assert torch.equal(out, ref_out), f"call {call}: output differs from fa_fwd_kvcache"
+        assert torch.equal(lse, ref_lse), f"call {call}: LSE differs from fa_fwd_kvcache"
+
+
+def test_noalloc_coarsens_the_split_until_the_partials_fit():
+    # 128 rows x 8 KV heads with capacity 2048: the usual 512-key split needs 4 partials per
+    # (row, KV head), 33.8 MB; 1024 keys still need 16.9 MB > 16 MiB, so the call runs one split
+    # of the whole capacity (8.5 MB) -- the split fa_fwd_kvcache takes with num_splits = 1
+    B, Hq, Hkv, D, cap = 128, 32, 8, 128, 2048
+    g = torch.Generator("cpu").manual_seed(40)
+    lengths = torch.randint(1, 200, (B,), generator=g).tolist()
+    lengths[3], lengths[77] = cap, 1500
+    w = W.kvcache(B, Hq, Hkv, D, cap, 0, 0, seed=41, lengths=lengths)
+    t = {n: x.cuda() for n, x in w.tensors.items()}
+    for _ in range(2):
+        out, lse = _noalloc(t, B, Hq, Hkv, cap, D, w.scale)
+        ref_out, ref_lse = _reference(t, B, Hq, Hkv, cap, D, w.scale, num_splits=1)
+        assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+    # and against the fp64 oracle on the rows' valid keys
+    L = max(lengths)
+    tt = w.tensors
+    o_ref, l_ref = oracle.kvcache_forward(H.f64(tt["q"]), H.f64(tt["k_cache"][:, :L]), H.f64(tt["v_cache"][:, :L]),
+                                          tt["cache_seqlens"].numpy(), w.scale, False)
+    H.check_o(out, o_ref)
+    H.check_lse(lse, l_ref)
+    assert np.isfinite(H.f64(out)).all()
 
 
 def test_noalloc_rejects_partials_beyond_the_fixed_array():
