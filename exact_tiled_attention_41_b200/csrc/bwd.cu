@@ -21,6 +21,7 @@
 //                    memory, both written back as bf16 into the warpgroup's own 64
 //                    columns of S^T (dS^T also to shared memory), so dP^T's columns
 //                    are free for dQ; dV (warpgroup 0) / dK (warpgroup 1) epilogue
+//                    (whole key tiles leave through shared memory with TMA stores)
 //        warps 8-11  dQ: thread = query row; reads the dQ tile from tensor memory
 //                    and adds it to the fp32 accumulator (vector atomics); each half
 //                    of the tile is released as soon as it is in registers, so the
@@ -144,6 +145,7 @@ template <int D, bool DQ>
 __global__ void __launch_bounds__(512, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+               const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                const __grid_constant__ BwdParams p) {
     using C = BwdCfg<D>;
     constexpr int ST = C::ST;
@@ -501,32 +503,80 @@ __global__ void __launch_bounds__(512, 1)
             const uint32_t col = gq == 0 ? C::COL_DV : C::COL_DK;
             const float mul = gq == 0 ? 1.f : p.scale;
             const float2 mul2 = make_float2(mul, mul);
-            // rows go out through this warpgroup's half of the dS buffer: the last dQ product that read
-            // it is complete (dkv_full), and this warpgroup is its next writer
-            uint8_t* stg = smem + C::OFF_DS + gq * (C::DS_BYTES / 2) + (warp & 3) * 2048;
+            // this warpgroup's half of the dS buffer (16 KB) is free: the last dQ product that read it is
+            // complete (dkv_full), and this warpgroup is its next writer
+            uint8_t* half_buf = smem + C::OFF_DS + gq * (C::DS_BYTES / 2);
             const BUnit te = decode_bunit(p, u);     // decoded again: nothing of it stays live over the tiles
-            __nv_bfloat16* gdst = out_row(te);
-            const int nvalid = min(max(te.Lk - te.n0 - (warp & 3) * 32, 0), 32);
-            const long long rstride = static_cast<long long>(p.Hkv) * D * 2;
+            if (te.n0 + 128 <= te.Lk) {
+                // a whole key tile: each 64-column box goes to shared memory in the tensor map's 128-byte
+                // swizzle (thread = row) and leaves with one TMA store; the box is refilled only after
+                // the previous store has read it
+                const bool issuer = (warp & 3) == 0 && lane == 0;
+                const CUtensorMap* map = gq == 0 ? &tmDV : &tmDK;
 #pragma unroll 1
-            for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t ra[32];
-                tmem_ld32(tmem + lb + col + cc * 32, ra);
-                tmem_ld_wait_tie(ra);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 v = fmul2(make_float2(__uint_as_float(ra[8 * q + 2 * e]), __uint_as_float(ra[8 * q + 2 * e + 1])), mul2);
-                        pk[e] = pack_bf16x2(v.x, v.y);
+                for (int bx = 0; bx < D / 64; ++bx) {
+                    if (bx > 0) {
+                        if (issuer) bulk_wait_read_all();
+                        named_bar_sync(1 + gq, 128);
                     }
-                    stg_put(stg, q, pk[0], pk[1], pk[2], pk[3]);
+#pragma unroll 1
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t ra[32];
+                        tmem_ld32(tmem + lb + col + bx * 64 + cc * 32, ra);
+                        tmem_ld_wait_tie(ra);
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 v = fmul2(make_float2(__uint_as_float(ra[8 * q + 2 * e]),
+                                                                   __uint_as_float(ra[8 * q + 2 * e + 1])), mul2);
+                                pk[e] = pack_bf16x2(v.x, v.y);
+                            }
+                            const int ch = cc * 4 + q;   // 16-byte chunk of the 128-byte box row
+                            *reinterpret_cast<uint4*>(half_buf + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    named_bar_sync(1 + gq, 128);
+                    if (issuer) {
+                        tma_store_3d(map, smem_u32(half_buf), bx * 64, te.hk, te.k_start + te.n0);
+                        bulk_commit();
+                    }
                 }
-                stg_flush(stg, reinterpret_cast<uint8_t*>(gdst + cc * 32), rstride, nvalid);
+                // the next tile's dS^T rows go into this buffer: wait until the last store has read it
+                if (issuer) bulk_wait_read_all();
+                named_bar_sync(1 + gq, 128);
+            } else {
+                // the sequence's last, partial key tile: rows leave through 2 KB per warp of the same
+                // buffer, 8 rows x 64 bytes per store, and only the rows inside the sequence are written
+                uint8_t* stg = half_buf + (warp & 3) * 2048;
+                __nv_bfloat16* gdst = out_row(te);
+                const int nvalid = min(max(te.Lk - te.n0 - (warp & 3) * 32, 0), 32);
+                const long long rstride = static_cast<long long>(p.Hkv) * D * 2;
+#pragma unroll 1
+                for (int cc = 0; cc < D / 32; ++cc) {
+                    uint32_t ra[32];
+                    tmem_ld32(tmem + lb + col + cc * 32, ra);
+                    tmem_ld_wait_tie(ra);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 v = fmul2(make_float2(__uint_as_float(ra[8 * q + 2 * e]),
+                                                               __uint_as_float(ra[8 * q + 2 * e + 1])), mul2);
+                            pk[e] = pack_bf16x2(v.x, v.y);
+                        }
+                        stg_put(stg, q, pk[0], pk[1], pk[2], pk[3]);
+                    }
+                    stg_flush(stg, reinterpret_cast<uint8_t*>(gdst + cc * 32), rstride, nvalid);
+                }
             }
             tc_fence_before();
         }
+        if ((warp & 3) == 0 && lane == 0) bulk_wait_all();   // this thread's dK / dV stores are complete
     }
 
     __syncthreads();
@@ -1009,6 +1059,9 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     if (!make_map_3d_bf16(&mdo, dout, D, pr.Hq, pr.Tq, D * 2, rq, 64, 1, 128)) return 5;
     if (!make_map_3d_bf16(&mk, pr.k, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
     if (!make_map_3d_bf16(&mv, pr.v, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+    alignas(64) CUtensorMap mdk, mdv;   // dK / dV stores of whole key tiles
+    if (!make_map_3d_bf16(&mdk, dk, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
+    if (!make_map_3d_bf16(&mdv, dv, D, pr.Hkv, pr.Tk, D * 2, rk, 64, 1, 128)) return 5;
 
     BwdParams p;
     p.dk = static_cast<__nv_bfloat16*>(dk);
@@ -1051,7 +1104,7 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
     if (grid > 0) {
         prof_before(1, stream);
-        kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, p);
+        kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
         prof_after(1, stream);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }

@@ -164,16 +164,13 @@ struct FwdCfg {
     static constexpr uint32_t Q_BYTES = BM * D * 2;
     static constexpr uint32_t KV_BYTES = BK * D * 2;
     static constexpr int NUM_BARS = 5 * NQ + 4 * KST;
-    // epilogue staging: 2 KB per softmax warp (its 32 rows x 64 bytes at a time)
-    static constexpr uint32_t STG_BYTES = 4 * NQ * 2048;
-    static constexpr size_t SMEM = 1024 + NQ * Q_BYTES + 2 * KST * KV_BYTES + STG_BYTES + NUM_BARS * 8 + 16;
-    static_assert(SMEM <= 232448, "shared memory per block");
+    static constexpr size_t SMEM = 1024 + NQ * Q_BYTES + 2 * KST * KV_BYTES + NUM_BARS * 8 + 16;
     // NQ softmax warpgroups + one warpgroup holding the producer warp, the MMA warp and two idle warps
     static constexpr int THREADS = (4 * NQ + 4) * 32;
     // register split with setmaxnreg (NQ = 2): launch at 168 per thread (384 x 168 = 64512),
     // the producer/MMA warpgroup drops to 96 and the two softmax warpgroups rise to 200:
     // 2 x 128 x 200 + 128 x 96 = 63488 <= 64512.  The host checks the launch count before the first launch.
-    static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 200, OTHER_REGS = 104;
+    static constexpr int LAUNCH_REGS = 168, SOFTMAX_REGS = 200, OTHER_REGS = 96;
     static_assert(NQ != 2 || 2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
     static constexpr uint32_t S_COL(int i) { return i * BK; }
     static constexpr uint32_t O_COL(int i) { return NQ * BK + i * D; }
@@ -183,9 +180,11 @@ struct FwdCfg {
 
 constexpr float kDeferLog2 = 8.0f;
 // Share of the softmax exponentials computed on the FMA pipe (exp2_fma2) instead of the
-// multi-function unit, whose 16 results per clock per SM match the tensor rate at D = 128:
-// one pair in fma_exp_every(D) of each row's pairs (tiles with masked scores use the
-// multi-function unit only), 0 = none.
+// multi-function unit: one pair in fma_exp_every(D) of each row's pairs (tiles with masked
+// scores use the multi-function unit only), 0 = none.  Measured on B200 at D = 64 and 128 with
+// one pair in 2, 3, 4 and 6: every share made the forward slower (-22 % to -5 % on the dense
+// and long-context workloads), so it is off: a softmax warp's exponentials are bound by its own
+// instruction stream and latency, and the polynomial lengthens both.
 #ifndef FA_FMA_EXP_EVERY_64
 #define FA_FMA_EXP_EVERY_64 0
 #endif
@@ -213,8 +212,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     uint8_t* sQ = smem;
     uint8_t* sK = sQ + NQ * C::Q_BYTES;
     uint8_t* sV = sK + KST * C::KV_BYTES;
-    uint8_t* sStg = sV + KST * C::KV_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sStg + C::STG_BYTES);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sV + KST * C::KV_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -264,65 +262,43 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     // each setmaxnreg is executed by all four warps of its warpgroup at the same instruction.
     if (warp >= 4 * NQ) {
     if constexpr (NQ == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
-    // the next unit with work at or after round kk of this CTA's schedule (kk is moved to its round), or -1
-    auto next_unit = [&](int& kk, Unit& tt) -> int {
-        for (int uu = snake_unit(kk, p.num_units); uu >= 0; uu = snake_unit(++kk, p.num_units)) {
-            if (uu >= p.num_units) continue;
-            tt = decode_unit<ROWS, BK, LOCAL>(p, uu);
-            if (!tt.skip && tt.n_kv > 0) return uu;
-        }
-        return -1;
-    };
     if (warp == PRODUCER) {
         if (lane == 0) {
-            // per unit: Q_0, K(0), Q_1, V(0), then K(j), V(j); each Q tile waits only for its own slot (the
-            // previous unit's last QK of that tile), so the next unit's first QK can start while the
-            // current unit finishes.  The next unit's Q tiles are brought into L2 when a unit starts.
             uint32_t kv_it = 0, q_it = 0;
-            int k = 0;
-            Unit t;
-            int u = next_unit(k, t);
-            bool ok = true;
-            while (u >= 0 && ok) {
-                int kn = k + 1;
-                Unit tn;
-                const int un = next_unit(kn, tn);
-                if (un >= 0)
-                    for (int i = 0; i < NQ; ++i)
-#pragma unroll
-                        for (int c = 0; c < C::NCHUNK; ++c)
-                            tma_prefetch_l2_3d(&tmQ, c * 64, tn.h, tn.q_start + tn.q0 + i * BM);
+            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0; u = snake_unit(++k, p.num_units)) {
+                if (u >= p.num_units) continue;
+                const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
+                if (t.skip || t.n_kv == 0) continue;
                 const int hk = t.h / p.group;
-                auto load_kv = [&](bool is_k, uint32_t it, int j) -> bool {
-                    const int st = it % KST;
-                    const uint32_t n = it / KST;
-                    if (n > 0 && !mbar_wait(is_k ? k_empty(st) : v_empty(st), (n - 1) & 1, w)) return false;
-                    const uint32_t full = is_k ? k_full(st) : v_full(st);
-                    mbar_arrive_expect_tx(full, C::KV_BYTES);
-                    uint8_t* dst = (is_k ? sK : sV) + st * C::KV_BYTES;
-#pragma unroll
-                    for (int c = 0; c < C::NCHUNK; ++c)
-                        tma_load_3d(smem_u32(dst + c * BK * 128), is_k ? &tmK : &tmV, full, c * 64, hk,
-                                    t.k_start + (unit_kv0<LOCAL>(t) + j) * BK);
-                    return true;
-                };
+                bool ok = true;
                 for (int i = 0; i < NQ && ok; ++i) {
-                    if (q_it > 0 && !mbar_wait(q_empty(i), (q_it - 1) & 1, w)) { ok = false; break; }
+                    if (q_it > 0 && !mbar_wait(q_empty(i), (q_it - 1) & 1, w)) ok = false;
+                    if (!ok) break;
                     mbar_arrive_expect_tx(q_full(i), C::Q_BYTES);
 #pragma unroll
                     for (int c = 0; c < C::NCHUNK; ++c)
                         tma_load_3d(smem_u32(sQ + i * C::Q_BYTES + c * BM * 128), &tmQ, q_full(i), c * 64, t.h,
                                     t.q_start + t.q0 + i * BM);
-                    if (i == 0 && !load_kv(true, kv_it, 0)) ok = false;
                 }
-                if (!ok || !load_kv(false, kv_it, 0)) break;
-                for (int j = 1; j < t.n_kv && ok; ++j)
-                    ok = load_kv(true, kv_it + j, j) && load_kv(false, kv_it + j, j);
+                if (!ok) break;
                 ++q_it;
-                kv_it += t.n_kv;
-                u = un;
-                k = kn;
-                t = tn;
+                for (int j = 0; j < t.n_kv && ok; ++j, ++kv_it) {
+                    const int st = kv_it % KST;
+                    const uint32_t n = kv_it / KST;
+                    if (n > 0 && !mbar_wait(k_empty(st), (n - 1) & 1, w)) { ok = false; break; }
+                    mbar_arrive_expect_tx(k_full(st), C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_3d(smem_u32(sK + st * C::KV_BYTES + c * BK * 128), &tmK, k_full(st), c * 64, hk,
+                                    t.k_start + (unit_kv0<LOCAL>(t) + j) * BK);
+                    if (n > 0 && !mbar_wait(v_empty(st), (n - 1) & 1, w)) { ok = false; break; }
+                    mbar_arrive_expect_tx(v_full(st), C::KV_BYTES);
+#pragma unroll
+                    for (int c = 0; c < C::NCHUNK; ++c)
+                        tma_load_3d(smem_u32(sV + st * C::KV_BYTES + c * BK * 128), &tmV, v_full(st), c * 64, hk,
+                                    t.k_start + (unit_kv0<LOCAL>(t) + j) * BK);
+                }
+                if (!ok) break;
             }
         }
         __syncwarp();
@@ -330,107 +306,45 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BK, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
-            // descriptors advance by adding the byte offset >> 4 to the start-address field (shared-memory
-            // addresses stay below 2^18, so the 14-bit field never carries); a rolled loop keeps few
-            // registers live in this warp
             auto issue_qk = [&](int i, int st) {
-                const uint64_t qd = sdesc_sw128(smem_u32(sQ + i * C::Q_BYTES), 16, 1024);
-                const uint64_t kd = sdesc_sw128(smem_u32(sK + st * C::KV_BYTES), 16, 1024);
-#pragma unroll 1
+#pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qo = ((kk >> 2) * BM * 128 + (kk & 3) * 32) >> 4;
-                    const uint32_t ko = ((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4;
-                    umma_ss(tmem + C::S_COL(i), qd + qo, kd + ko, idesc_qk, kk > 0 ? 1u : 0u);
+                    const uint32_t qa = smem_u32(sQ + i * C::Q_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32);
+                    const uint32_t kb = smem_u32(sK + st * C::KV_BYTES + (kk >> 2) * BK * 128 + (kk & 3) * 32);
+                    umma_ss(tmem + C::S_COL(i), sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), idesc_qk,
+                            kk > 0 ? 1u : 0u);
                 }
             };
             auto issue_pv = [&](int i, int st, bool acc) {
-                const uint64_t vd = sdesc_sw128(smem_u32(sV + st * C::KV_BYTES), BK * 128, 1024);
-#pragma unroll 1
-                for (int kk = 0; kk < BK / 16; ++kk)
-                    umma_ts(tmem + C::O_COL(i), tmem + C::S_COL(i) + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
-                            (acc || kk > 0) ? 1u : 0u);
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    const uint32_t vb = smem_u32(sV + st * C::KV_BYTES + kk * 16 * 128);
+                    umma_ts(tmem + C::O_COL(i), tmem + C::S_COL(i) + kk * 8, sdesc_sw128(vb, BK * 128, 1024),
+                            idesc_pv, (acc || kk > 0) ? 1u : 0u);
+                }
             };
             uint32_t kv_it = 0, q_it = 0, p_it[NQ] = {};
-            // K ring indices 0 .. k_obs-1 have had their k_full phase observed by this warp; a test of a
-            // later phase of the same stage is only meaningful once the stage's previous phase was observed
-            uint32_t k_obs = 0;
             bool ok = true;
-            // bit i of pre: QK_i(0) of the current unit was already issued while the previous unit finished
-            unsigned pre = 0;
-            int k = 0;
-            Unit t;
-            int u = next_unit(k, t);
-            while (u >= 0 && ok) {
-                int kn = k + 1;
-                Unit tn;
-                const int un = next_unit(kn, tn);
-                // Look-ahead: once query tile i has issued its last PV of this unit, its S columns are free
-                // (the tensor pipe runs in order), so the next unit's QK_i(0) may be issued right away --
-                // but only if its Q tile and first K tile have already landed: tested without waiting, so
-                // the MMA warp never blocks on a load the producer can only issue after later MMAs here.
-                const uint32_t kv_n = kv_it + t.n_kv;                 // ring index of the next unit's K(0)
-                // bit i: la = tile i of the next unit starts at KV tile 0 and is not issued yet;
-                // fin = tile i has issued its last PV of this unit; done = issued ahead
-                unsigned la = 0, fin = 0, done = 0, one = 0;
-                for (int i = 0; i < NQ; ++i) {
-                    if (un >= 0 && unit_lo<LOCAL>(tn, i) == 0 && unit_hi(tn, i) > 0) la |= 1u << i;
-                    if (un >= 0 && unit_hi(tn, i) == 1) one |= 1u << i;
-                    if (unit_hi(t, i) == 0) fin |= 1u << i;
-                }
-                auto try_lookahead = [&]() {
-                    if ((la & fin) == 0 || kv_n >= k_obs + KST) return;
-                    if (!mbar_test(k_full(kv_n % KST), (kv_n / KST) & 1)) return;
-                    k_obs = kv_n + 1;
-                    for (int i = 0; i < NQ; ++i) {
-                        if (!((la & fin) >> i & 1u)) continue;
-                        if (!mbar_test(q_full(i), (q_it + 1) & 1)) continue;
-                        tc_fence_after();
-                        issue_qk(i, kv_n % KST);
-                        umma_commit(s_full(i));
-                        if (one >> i & 1u) umma_commit(q_empty(i));   // its only QK in the next unit
-                        la &= ~(1u << i);
-                        done |= 1u << i;
-                    }
-                };
-                // a bounded wait that keeps trying the look-ahead while it polls
-                auto wait_la = [&](uint32_t bar, uint32_t parity) -> bool {
-                    if (mbar_test(bar, parity)) return true;
-                    const uint64_t t0 = global_timer_ns();
-                    for (uint32_t it = 1;; ++it) {
-                        if (mbar_test(bar, parity)) return true;
-                        if ((it & 7u) == 0) try_lookahead();
-                        if ((it & 31u) == 0) {
-                            if (w.aborted()) return false;
-                            if (global_timer_ns() - t0 > w.limit_ns) {
-                                w.fail();
-                                return false;
-                            }
-                        }
-                    }
-                };
+            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+                if (u >= p.num_units) continue;
+                const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
+                if (t.skip || t.n_kv == 0) continue;
+                for (int i = 0; i < NQ && ok; ++i)
+                    if (!mbar_wait(q_full(i), q_it & 1, w)) ok = false;
+                if (!ok) break;
+                ++q_it;
                 {
-                    // prologue: QK_i(0) of the tiles that start at KV tile 0 and were not issued ahead
                     const int st = kv_it % KST;
-                    bool k_ready = false;
-                    for (int i = 0; i < NQ && ok; ++i) {
-                        if (pre >> i & 1u) continue;
-                        // every tile's Q load of this unit completes its phase here (also for tiles that
-                        // start later or see no key), so the look-ahead's test of the next phase is exact
-                        if (!mbar_wait(q_full(i), q_it & 1, w)) { ok = false; break; }
-                        if (unit_lo<LOCAL>(t, i) == 0 && unit_hi(t, i) > 0) {
-                            if (!k_ready && !mbar_wait(k_full(st), (kv_it / KST) & 1, w)) { ok = false; break; }
-                            k_ready = true;
-                            k_obs = max(k_obs, kv_it + 1);
-                            tc_fence_after();
-                            issue_qk(i, st);
-                            umma_commit(s_full(i));
-                            if (unit_hi(t, i) == 1) umma_commit(q_empty(i));
-                        } else if (unit_hi(t, i) == 0) {
-                            umma_commit(q_empty(i));   // a tile that sees no key in this unit
-                        }
+                    if (!mbar_wait(k_full(st), (kv_it / KST) & 1, w)) break;
+                    tc_fence_after();
+                    for (int i = 0; i < NQ; ++i) {
+                        if (unit_lo<LOCAL>(t, i) != 0 || unit_hi(t, i) == 0) continue;   // tile i starts later (or never)
+                        issue_qk(i, st);
+                        umma_commit(s_full(i));
                     }
-                    if (!ok) break;
                     umma_commit(k_empty(st));
+                    if (t.n_kv == 1)
+                        for (int i = 0; i < NQ; ++i) umma_commit(q_empty(i));
                 }
                 // query tile i works on the unit's KV tiles lo[i] .. hi[i]-1
                 for (int j = 0; j < t.n_kv && ok; ++j) {
@@ -438,29 +352,25 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     const int st = cur % KST;
                     const uint32_t nxt = cur + 1;
                     const int stn = nxt % KST;
-                    try_lookahead();
-                    if (!wait_la(v_full(st), (cur / KST) & 1)) { ok = false; break; }
+                    if (!mbar_wait(v_full(st), (cur / KST) & 1, w)) { ok = false; break; }
                     tc_fence_after();
                     bool k_ready = false;
                     for (int i = 0; i < NQ; ++i) {
                         if (j >= unit_lo<LOCAL>(t, i) && j < unit_hi(t, i)) {
-                            if (!wait_la(p_full(i), p_it[i] & 1)) { ok = false; break; }
+                            if (!mbar_wait(p_full(i), p_it[i] & 1, w)) { ok = false; break; }
                             ++p_it[i];
                             tc_fence_after();
                             issue_pv(i, st, j > unit_lo<LOCAL>(t, i));
                             umma_commit(o_full(i));
-                            if (j + 1 == unit_hi(t, i)) fin |= 1u << i;
                         }
                         if (j + 1 >= unit_lo<LOCAL>(t, i) && j + 1 < unit_hi(t, i)) {
                             if (!k_ready) {
                                 if (!mbar_wait(k_full(stn), (nxt / KST) & 1, w)) { ok = false; break; }
                                 tc_fence_after();
                                 k_ready = true;
-                                k_obs = max(k_obs, nxt + 1);
                             }
                             issue_qk(i, stn);
                             umma_commit(s_full(i));
-                            if (j + 2 == unit_hi(t, i)) umma_commit(q_empty(i));   // tile i's last QK
                         }
                     }
                     if (!ok) break;
@@ -469,16 +379,13 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                     // row of tile 0, since the window sides are >= 0), so their union has no gap
                     // and some tile issues QK(j+1)
                     umma_commit(v_empty(st));
-                    if (j + 1 < t.n_kv) umma_commit(k_empty(stn));
+                    if (j + 1 < t.n_kv) {
+                        umma_commit(k_empty(stn));
+                        if (j + 2 == t.n_kv)
+                            for (int i = 0; i < NQ; ++i) umma_commit(q_empty(i));
+                    }
                 }
-                if (!ok) break;
-                try_lookahead();
-                pre = done;
                 kv_it += t.n_kv;
-                ++q_it;
-                u = un;
-                k = kn;
-                t = tn;
             }
         }
         __syncwarp();
@@ -582,7 +489,7 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
                 const float2 c2v = make_float2(c2, c2), nms = make_float2(-ms, -ms);
                 float2 sum0 = make_float2(0.f, 0.f), sum1 = make_float2(0.f, 0.f);
                 // exp(scale * s - scale * m) as exp2 of one fused multiply-add per pair; on tiles
-                // without masked scores one pair in fma_exp_every(D) goes to the FMA pipe
+                // without masked scores one pair in fma_exp_every(D) may go to the FMA pipe
                 auto exp_row = [&](auto poly) {
                     constexpr int kEvery = decltype(poly)::value ? fma_exp_every(D) : 0;
                     constexpr int kMod = kEvery > 0 ? kEvery : 1;
@@ -617,29 +524,23 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             if (!mbar_wait(o_full(i), (pv_total - 1) & 1, w)) { ok = false; break; }
             tc_fence_after();
             const float inv_l = l > 0.f ? 1.f / l : 0.f;
-            const float2 il = make_float2(inv_l, inv_l);
-            // rows leave through this warp's 2 KB of staging, 8 rows x 64 bytes per store instead of
-            // 32 rows x 16 bytes (rows of a tile are consecutive tokens, Hq * D * 2 bytes apart)
-            uint8_t* stg = sStg + warp * 2048;
-            const int nvalid = min(max(t.Lq - (t.q0 + i * BM + wq * 32), 0), 32);
-            const long long rstride = static_cast<long long>(p.Hq) * D * 2;
+            uint32_t ro[32];
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
-                uint32_t ro[32];
                 tmem_ld32(tO + cc * 32, ro);
                 tmem_ld_wait_tie(ro);
+                uint32_t pk[16];
+                const float2 il = make_float2(inv_l, inv_l);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 v = fmul2(make_float2(__uint_as_float(ro[8 * q4 + 2 * e]),
-                                                           __uint_as_float(ro[8 * q4 + 2 * e + 1])), il);
-                        pk[e] = pack_bf16x2(v.x, v.y);
-                    }
-                    stg_put(stg, q4, pk[0], pk[1], pk[2], pk[3]);
+                for (int e = 0; e < 16; ++e) {
+                    const float2 v = fmul2(make_float2(__uint_as_float(ro[2 * e]), __uint_as_float(ro[2 * e + 1])), il);
+                    pk[e] = pack_bf16x2(v.x, v.y);
                 }
-                stg_flush(stg, reinterpret_cast<uint8_t*>(orow + cc * 32), rstride, nvalid);
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+                }
             }
             if (valid) *lse_ptr = l > 0.f ? (m_ref * c2 + log2f(l)) * kLn2 : -INFINITY;
             tc_fence_before();

@@ -16,8 +16,17 @@ row rise (or fall) by a set amount from one 128-key tile to the next:
     with rising rows inside every warp.
 
 Each case is checked against the fp64 oracle (forward O, LSE, and the backward, which
-recomputes P from the LSE) at the stated tolerances, and a numpy model of the tiled loop
-with the O rescale left out shows that such a slip would miss those tolerances by far.
+recomputes P from the LSE), and a numpy model of the tiled loop with the O rescale left out
+shows that such a slip would miss the O tolerance by far.
+
+Tolerances: LSE (1e-3) and the gradients (2e-2) as stated for the method.  The O bound of
+1e-2 is stated for N(0, 1) inputs, whose softmax is flat and whose O is small; these inputs
+make each row's softmax peaked (|O| up to about 3).  The kernel rounds every P to bf16 before
+the PV product -- including the dominant terms, which under the deferred reference max are up
+to 2^8 rather than exactly 1 -- and rounds O to bf16, so an element of O may be off by
+2^-9 (max_j |v_j| + |O|) <= 2^-8 max |V|; the O tolerance here is that bound (plus 1e-3 for
+fp32 accumulation) or 1e-2, whichever is larger.  A float32 model of the tiled loop with the
+deferred max reproduces the kernel's largest O error on these inputs to the last digit.
 """
 
 import math
@@ -74,6 +83,10 @@ def _varlen_case(D, causal, rise_log2, seed):
     return w
 
 
+def _o_tol(w):
+    return max(H.O_TOL, 2.0 ** -8 * float(w.tensors["v"].float().abs().max()) + 1e-3)
+
+
 def _skip_rescale_model(qh, kh, vh, scale, causal):
     """Tiled online softmax of one head (fp64) with the O rescale left out: O keeps the
     contributions of earlier tiles at their old reference while l is rescaled."""
@@ -102,14 +115,14 @@ def _skip_rescale_model(qh, kh, vh, scale, causal):
 @pytest.mark.parametrize("rise_log2", [9.0, 3.0])
 def test_dense_rising_scores(D, causal, rise_log2):
     w = _dense_case(D, causal, rise_log2, seed=D + 10 * causal + int(rise_log2))
-    H.check_dense(w)
+    H.check_dense(w, o_tol=_o_tol(w))
     if rise_log2 > 8.0:
         # the inputs make the rescale matter: leaving it out would be far outside the tolerance
         t = w.tensors
         qh, kh, vh = H.f64(t["q"][0, :, 0]), H.f64(t["k"][0, :, 0]), H.f64(t["v"][0, :, 0])
         o_ref, _ = oracle.mha_forward(H.f64(t["q"]), H.f64(t["k"]), H.f64(t["v"]), w.scale, causal)
         bad = _skip_rescale_model(qh, kh, vh, w.scale, causal)
-        assert np.abs(bad - o_ref[0, :, 0]).max() > 10 * H.O_TOL
+        assert np.abs(bad - o_ref[0, :, 0]).max() > 10 * _o_tol(w)
 
 
 @pytest.mark.parametrize("D", [64, 128, 256])
@@ -117,10 +130,10 @@ def test_dense_rising_scores(D, causal, rise_log2):
 @pytest.mark.parametrize("rise_log2", [9.0, 3.0])
 def test_varlen_rising_scores(D, causal, rise_log2):
     w = _varlen_case(D, causal, rise_log2, seed=7 * D + causal + int(rise_log2))
-    H.check_varlen(w)
+    H.check_varlen(w, o_tol=_o_tol(w))
 
 
 @pytest.mark.parametrize("rise_log2", [9.0, 3.0])
 def test_rising_scores_deterministic_backward(rise_log2):
     w = _dense_case(128, True, rise_log2, seed=77)
-    H.check_dense(w, deterministic=True)
+    H.check_dense(w, deterministic=True, o_tol=_o_tol(w))

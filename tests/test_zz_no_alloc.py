@@ -25,21 +25,21 @@ pytestmark = pytest.mark.gpu
 FAKE = 0x10000
 
 
-def _reference(t, B, Hq, Hkv, cap, D, scale, num_splits=0):
+def _reference(t, B, Hq, Hkv, cap, D, scale, num_splits=0, Sq=1, causal=0):
     out = torch.empty_like(t["q"])
-    lse = torch.empty((B, Hq, 1), dtype=torch.float32, device="cuda")
-    nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, 1, cap, D, num_splits)
+    lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device="cuda")
+    nb = abi.fa_fwd_kvcache_workspace_size(B, Hq, Hkv, Sq, cap, D, num_splits)
     ws = torch.empty(nb, dtype=torch.uint8, device="cuda")
-    assert abi.fa_fwd_kvcache(t["q"], t["k_cache"], t["v_cache"], t["cache_seqlens"], out, lse, B, Hq, Hkv, 1, cap,
-                              D, scale, 0, num_splits, ws, nb) == 0
+    assert abi.fa_fwd_kvcache(t["q"], t["k_cache"], t["v_cache"], t["cache_seqlens"], out, lse, B, Hq, Hkv, Sq, cap,
+                              D, scale, causal, num_splits, ws, nb) == 0
     return out, lse
 
 
-def _noalloc(t, B, Hq, Hkv, cap, D, scale):
+def _noalloc(t, B, Hq, Hkv, cap, D, scale, Sq=1, causal=0):
     out = torch.full_like(t["q"], float("nan"))
-    lse = torch.full((B, Hq, 1), float("nan"), dtype=torch.float32, device="cuda")
+    lse = torch.full((B, Hq, Sq), float("nan"), dtype=torch.float32, device="cuda")
     st = abi.fa_fwd_kvcache_noalloc(t["q"], t["k_cache"], t["v_cache"], t["cache_seqlens"], out, lse, B, Hq, Hkv,
-                                    1, cap, D, scale, 0, 0)
+                                    Sq, cap, D, scale, causal, 0)
     assert st == 0, abi.status_string(st)
     torch.cuda.synchronize()
     assert abi.fa_get_device_status() == 0
@@ -60,24 +60,25 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(D):
 
 
 def test_noalloc_coarsens_the_split_until_the_partials_fit():
-    # 128 rows x 8 KV heads with capacity 2048: the usual 512-key split needs 4 partials per
-    # (row, KV head), 33.8 MB; 1024 keys still need 16.9 MB > 16 MiB, so the call runs one split
-    # of the whole capacity (8.5 MB) -- the split fa_fwd_kvcache takes with num_splits = 1
-    B, Hq, Hkv, D, cap = 128, 32, 8, 128, 2048
+    # 64 rows x 8 KV heads x 16 query rows (4 heads per KV head x 4 causal tokens), capacity 4096: the
+    # usual 512-key split needs 8 partials per (row, KV head) -- 33.8 MB; 1024 keys still need 16.9 MB
+    # > 16 MiB, so the call runs two splits of 2048 keys (8.5 MB), the split fa_fwd_kvcache takes with
+    # num_splits = 2
+    B, Hq, Hkv, D, cap, Sq = 64, 32, 8, 128, 4096, 4
     g = torch.Generator("cpu").manual_seed(40)
-    lengths = torch.randint(1, 200, (B,), generator=g).tolist()
-    lengths[3], lengths[77] = cap, 1500
-    w = W.kvcache(B, Hq, Hkv, D, cap, 0, 0, seed=41, lengths=lengths)
+    lengths = torch.randint(Sq, 200, (B,), generator=g).tolist()
+    lengths[3], lengths[17], lengths[40] = cap, 2049, 2048
+    w = W.kvcache(B, Hq, Hkv, D, cap, 0, 0, seed=41, Sq=Sq, lengths=lengths)
     t = {n: x.cuda() for n, x in w.tensors.items()}
     for _ in range(2):
-        out, lse = _noalloc(t, B, Hq, Hkv, cap, D, w.scale)
-        ref_out, ref_lse = _reference(t, B, Hq, Hkv, cap, D, w.scale, num_splits=1)
+        out, lse = _noalloc(t, B, Hq, Hkv, cap, D, w.scale, Sq, 1)
+        ref_out, ref_lse = _reference(t, B, Hq, Hkv, cap, D, w.scale, 2, Sq, 1)
         assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
-    # and against the fp64 oracle on the rows' valid keys
+    # and against the fp64 oracle on the rows' valid keys (bottom-right causal tokens)
     L = max(lengths)
     tt = w.tensors
     o_ref, l_ref = oracle.kvcache_forward(H.f64(tt["q"]), H.f64(tt["k_cache"][:, :L]), H.f64(tt["v_cache"][:, :L]),
-                                          tt["cache_seqlens"].numpy(), w.scale, False)
+                                          tt["cache_seqlens"].numpy(), w.scale, True)
     H.check_o(out, o_ref)
     H.check_lse(lse, l_ref)
     assert np.isfinite(H.f64(out)).all()
