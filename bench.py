@@ -293,31 +293,59 @@ def run_ours(args, rank, world, local_rank):
     value = aggregate_tflops(step_flops, world, ms_per_step)
 
     # ----------------------------------------------------------------- end to end through the public API
+    # Each step copies its inputs from pinned host memory, runs the forward and backward through the
+    # torch-level API and copies every result back.  Three streams (copy in, compute, copy out) with
+    # two buffer sets: step i's results go out while step i+1's inputs come in (the two directions of
+    # the host link are independent); every dependency is an event.
     e2e_steps = min(args.steps, 30)
     pin = {n: x.cpu().pin_memory() for n, x in w.tensors.items()}
-    host_out = {n: torch.empty(x.shape, dtype=x.dtype, pin_memory=True)
-                for n, x in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    names_out = ("out", "lse", "dq", "dk", "dv")
+    shapes_out = {"out": (q.shape, q.dtype), "lse": (lse.shape, lse.dtype), "dq": (q.shape, q.dtype),
+                  "dk": (k.shape, k.dtype), "dv": (v.shape, v.dtype)}
+    host_out = [{n: torch.empty(sh, dtype=dt, pin_memory=True) for n, (sh, dt) in shapes_out.items()}
+                for _ in range(2)]
+    dev_in = [{n: torch.empty_like(x, device=dev) for n, x in pin.items()} for _ in range(2)]
     h2d = sum(x.numel() * x.element_size() for x in pin.values())
-    d2h = sum(x.numel() * x.element_size() for x in host_out.values())
+    d2h = sum(x.numel() * x.element_size() for x in host_out[0].values())
+    s_in, s_cmp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    started = [False, False]
 
-    def e2e_step():
-        dq_ = {n: x.to(dev, non_blocking=True) for n, x in pin.items()}
-        o_, l_ = A.flash_attn_func(dq_["q"], dq_["k"], dq_["v"], scale, True)
-        g = A.flash_attn_backward(dq_["do"], dq_["q"], dq_["k"], dq_["v"], o_, l_, scale, True,
-                                  deterministic=bool(det))
-        for n, x in zip(("out", "lse", "dq", "dk", "dv"), (o_, l_) + tuple(g)):
-            host_out[n].copy_(x, non_blocking=True)
+    def e2e_step(i):
+        b_ = i % 2
+        x = dev_in[b_]
+        with torch.cuda.stream(s_in):
+            if started[b_]:
+                s_in.wait_event(ev_cmp[b_])          # the compute of step i-2 has read this buffer set
+            for n, src in pin.items():
+                x[n].copy_(src, non_blocking=True)
+            ev_in[b_].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[b_])
+            o_, l_ = A.flash_attn_func(x["q"], x["k"], x["v"], scale, True)
+            g = A.flash_attn_backward(x["do"], x["q"], x["k"], x["v"], o_, l_, scale, True,
+                                      deterministic=bool(det))
+            outs = (o_, l_) + tuple(g)
+            for t_ in outs:
+                t_.record_stream(s_out)              # the allocator keeps them until the copy-out is done
+            ev_cmp[b_].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[b_])
+            for n, t_ in zip(names_out, outs):
+                host_out[b_][n].copy_(t_, non_blocking=True)
+        started[b_] = True
 
-    for _ in range(3):
-        e2e_step()
+    for i in range(3):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(e2e_steps):
+        e2e_step(3 + i)
+    e1.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, world, dev)
     e2e_value = aggregate_tflops(step_flops, world, e2e_ms)
@@ -363,7 +391,10 @@ def run_ours(args, rank, world, local_rank):
             "step_frac_of_measured_peak": value / world / peak_t,
         },
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms, "api": "attention.flash_attn_func + flash_attn_backward, pinned host buffers"},
+                "ms_per_step": e2e_ms,
+                "api": "attention.flash_attn_func + flash_attn_backward, pinned host buffers; copy-in, compute and "
+                       "copy-out on three streams, two buffer sets (step i's results leave while step i+1's "
+                       "inputs arrive)"},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
@@ -525,6 +556,10 @@ def measure_extras(torch, abi, A, W, dev, pk):
     return res
 
 
+def w_scale(D):
+    return 1.0 / math.sqrt(D)
+
+
 def run_profile_case(args):
     """One mid-size case of a single path, for an ncu capture: inputs larger than L2 but under a GB."""
     import torch
@@ -546,6 +581,56 @@ def run_profile_case(args):
         fn = lambda: abi.fa_fwd_kvcache(t["q"], t["k_cache"], t["v_cache"], lens, out, lse, B, Hq, Hkv, 1, cap, D,
                                         w.scale, 0, 0, ws, nb, stream)
         name = "decode_B64_Hq32_Hkv8_cap2048_D128"
+    elif args.profile_case in ("varlen64", "varlen256"):
+        # the varlen packed workload (16 sequences, L ~ U[128, 4096], H = 16, causal): forward + backward
+        D = 64 if args.profile_case == "varlen64" else 256
+        w = W.varlen_packed(D, seed=0)
+        t = {n: x.to(dev) for n, x in w.tensors.items()}
+        m = w.meta
+        n, T, H = m["num_seqs"], m["total_q"], m["Hq"]
+        out = torch.empty_like(t["q"])
+        lse = torch.empty((H, T), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
+        nb = abi.fa_varlen_bwd_workspace_size(n, T, T, H, H, D)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        lens = (t["cu_q"][1:] - t["cu_q"][:-1]).cpu().double()
+        nbytes = 3.5 * float((4.0 * H * D * lens * lens * 0.5).sum())    # algorithmic FLOPs (fwd + bwd)
+
+        def fn():
+            st = abi.fa_varlen_fwd(t["q"], t["k"], t["v"], out, lse, t["cu_q"], t["cu_k"], n, m["max_q"], m["max_k"],
+                                   T, T, H, H, D, w.scale, 1, None, 0, stream)
+            return st | abi.fa_varlen_bwd(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, t["cu_q"], t["cu_k"],
+                                          n, m["max_q"], m["max_k"], T, T, H, H, D, w.scale, 1, ws, nb, stream)
+        name = f"varlen_16seq_L128-4096_H16_D{D}_causal_fwd+bwd"
+    elif args.profile_case in ("append", "decode256"):
+        # paged cache, B=64, Hq=32, Hkv=8, lengths uniform in [1024, 2048], pages of 256 keys; "append" adds 4
+        # causal query tokens whose k / v are written into the cache first, "decode256" is one token at D = 256
+        D = 128 if args.profile_case == "append" else 256
+        Sq = 4 if args.profile_case == "append" else 1
+        B, Hq, Hkv, cap, page = 64, 32, 8, 2304, 256
+        g = torch.Generator("cpu").manual_seed(5)
+        lens_l = torch.randint(1024, 2049, (B,), generator=g).tolist()
+        gd = torch.Generator(str(dev)).manual_seed(5)
+        nblk = B * cap // page
+        perm = torch.randperm(nblk, generator=g).reshape(B, cap // page).to(torch.int32).to(dev)
+        kc = torch.randn((nblk, page, Hkv, D), generator=gd, device=dev).to(torch.bfloat16)
+        vc = torch.randn((nblk, page, Hkv, D), generator=gd, device=dev).to(torch.bfloat16)
+        q_ = torch.randn((B, Sq, Hq, D), generator=gd, device=dev).to(torch.bfloat16)
+        kn = torch.randn((B, Sq, Hkv, D), generator=gd, device=dev).to(torch.bfloat16) if Sq > 1 else None
+        vn = torch.randn((B, Sq, Hkv, D), generator=gd, device=dev).to(torch.bfloat16) if Sq > 1 else None
+        lens = torch.tensor(lens_l, dtype=torch.int32, device=dev)
+        out = torch.empty_like(q_)
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+        nb = abi.fa_fwd_kvcache_ex_workspace_size(B, Hq, Hkv, Sq, D, page, cap // page, 0)
+        ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        keys = float(sum(lens_l)) + (B * Sq if Sq > 1 else 0)
+        nbytes = keys * Hkv * D * 2 * 2 + 2 * q_.numel() * 2 + (2 * 2 * B * Sq * Hkv * D * 2 if Sq > 1 else 0)
+        # the appended rows land at the same positions every call (cache_seqlens is not advanced)
+        fn = lambda: abi.fa_fwd_kvcache_ex(q_, kc, vc, lens, kn, vn, Sq if Sq > 1 else 0, None, perm, cap // page, nblk,
+                                           page, out, lse, B, Hq, Hkv, Sq, D, w_scale(D), 1, -1, -1, 0, ws, nb,
+                                           stream)
+        name = (f"decode_append4_paged256_B64_Hq32_Hkv8_L1024-2048_D{D}" if Sq > 1
+                else f"decode_paged256_B64_Hq32_Hkv8_L1024-2048_D{D}")
     else:
         C, B, S, H, D = 4, 2, 8192, 32, 128
         g = torch.Generator(str(dev)).manual_seed(3)
@@ -567,7 +652,10 @@ def run_profile_case(args):
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / max(args.steps, 1)
-    print(json.dumps({"profile_case": name, "ms": ms, "gbs": nbytes / ms / 1e6, "algorithmic_bytes": nbytes}))
+    if args.profile_case.startswith("varlen"):
+        print(json.dumps({"profile_case": name, "ms": ms, "tflops": nbytes / ms / 1e9, "algorithmic_flops": nbytes}))
+    else:
+        print(json.dumps({"profile_case": name, "ms": ms, "gbs": nbytes / ms / 1e6, "algorithmic_bytes": nbytes}))
     return 0
 
 
@@ -582,7 +670,8 @@ def main():
                     help="time the step with the deterministic backward (dq from the query-tile-stationary pass)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
-    ap.add_argument("--profile-case", choices=["decode", "merge"], default=None,
+    ap.add_argument("--profile-case", choices=["decode", "merge", "varlen64", "varlen256", "append", "decode256"],
+                    default=None,
                     help="run only a mid-size case of one path (inputs > L2, < 1 GB), e.g. under ncu, and print its time")
     args = ap.parse_args()
     if args.warmup < 3:

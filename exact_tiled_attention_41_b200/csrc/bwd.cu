@@ -150,8 +150,8 @@ __global__ void __launch_bounds__(512, 1)
     using C = BwdCfg<D>;
     constexpr int ST = C::ST;
     extern __shared__ __align__(1024) uint8_t smem[];
-    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);          // [ST][128]
-    float* sDel = sLSE + ST * 128;                                       // [ST][128]
+    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);          // [ST][128], -LSE2
+    float* sDel = sLSE + ST * 128;                                       // [ST][128], -Delta
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -233,8 +233,9 @@ __global__ void __launch_bounds__(512, 1)
                         const int row = m0 + qi;
                         const bool in = row < t.Lq;
                         const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
-                        sLSE[st * 128 + qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
-                        sDel[st * 128 + qi] = in ? __ldg(p.delta + idx) : 0.f;
+                        // stored negated, so the gradient step adds them (no negation per element)
+                        sLSE[st * 128 + qi] = in ? -__ldg(p.lse2 + idx) : -INFINITY;
+                        sDel[st * 128 + qi] = in ? -__ldg(p.delta + idx) : 0.f;
                     }
                     if (lane == 0) {
                         mbar_arrive_expect_tx(q_full(st), 2 * C::T_BYTES);
@@ -467,14 +468,14 @@ __global__ void __launch_bounds__(512, 1)
                             const float dla = x == 0 ? d4.x : d4.z, dlb = x == 0 ? d4.y : d4.w;
                             const float2 sv = make_float2(__uint_as_float(sh[e + x]), __uint_as_float(sh[e + x + 1]));
                             const float2 dv = make_float2(__uint_as_float(dh[e + x]), __uint_as_float(dh[e + x + 1]));
-                            const float2 a = ffma2(sv, c2v, make_float2(-la, -lbv));
+                            const float2 a = ffma2(sv, c2v, make_float2(la, lbv));
                             float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
                             if (any_mask) {
                                 const int qc = 64 * gq + half * 32 + e + x;
                                 pr.x = (qc >= qmin && qc <= qmax) ? pr.x : 0.f;
                                 pr.y = (qc + 1 >= qmin && qc + 1 <= qmax) ? pr.y : 0.f;
                             }
-                            const float2 ds = fmul2(pr, fadd2(dv, make_float2(-dla, -dlb)));
+                            const float2 ds = fmul2(pr, fadd2(dv, make_float2(dla, dlb)));
                             pp[(e + x) / 2] = pack_bf16x2(pr.x, pr.y);
                             dd[(e + x) / 2] = pack_bf16x2(ds.x, ds.y);
                         }
@@ -635,8 +636,8 @@ __global__ void __launch_bounds__(384, 1)
     constexpr int D = C::D;
     constexpr int ST = C::ST;
     extern __shared__ __align__(1024) uint8_t smem[];
-    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);          // [ST][64]
-    float* sDel = sLSE + ST * 64;                                        // [ST][64]
+    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);          // [ST][64], -LSE2
+    float* sDel = sLSE + ST * 64;                                        // [ST][64], -Delta
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -724,8 +725,9 @@ __global__ void __launch_bounds__(384, 1)
                             const int row = row0 + qi;
                             const bool in = row < t.Lq;
                             const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
-                            sLSE[st * 64 + qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
-                            sDel[st * 64 + qi] = in ? __ldg(p.delta + idx) : 0.f;
+                            // stored negated, so the gradient step adds them (no negation per element)
+                            sLSE[st * 64 + qi] = in ? -__ldg(p.lse2 + idx) : -INFINITY;
+                            sDel[st * 64 + qi] = in ? -__ldg(p.delta + idx) : 0.f;
                         }
                         if (lane == 0) {
                             mbar_arrive_expect_tx(q_full(st), 2 * C::IT_BYTES);
@@ -875,14 +877,14 @@ __global__ void __launch_bounds__(384, 1)
                                 const float dla = x == 0 ? d4.x : d4.z, dlb = x == 0 ? d4.y : d4.w;
                                 const float2 sv = make_float2(__uint_as_float(sh[e + x]), __uint_as_float(sh[e + x + 1]));
                                 const float2 dv = make_float2(__uint_as_float(dh[e + x]), __uint_as_float(dh[e + x + 1]));
-                                const float2 a = ffma2(sv, c2v, make_float2(-la, -lbv));
+                                const float2 a = ffma2(sv, c2v, make_float2(la, lbv));
                                 float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
                                 if (any_mask) {
                                     const int qc = half * 32 + e + x;
                                     pr.x = (qc >= qmin && qc <= qmax) ? pr.x : 0.f;
                                     pr.y = (qc + 1 >= qmin && qc + 1 <= qmax) ? pr.y : 0.f;
                                 }
-                                const float2 ds = fmul2(pr, fadd2(dv, make_float2(-dla, -dlb)));
+                                const float2 ds = fmul2(pr, fadd2(dv, make_float2(dla, dlb)));
                                 pp[(e + x) / 2] = pack_bf16x2(pr.x, pr.y);
                                 dd[(e + x) / 2] = pack_bf16x2(ds.x, ds.y);
                             }

@@ -306,22 +306,23 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_qk = idesc_bf16_f32(BM, BK, false, false);
             constexpr uint32_t idesc_pv = idesc_bf16_f32(BM, D, false, true);
+            // each product's descriptors are formed once and advanced by constant byte offsets >> 4 in the
+            // start-address field (shared-memory addresses stay below 2^18, so the 14-bit field never
+            // carries): two adds per MMA, so the issuer keeps up with the tensor pipe
             auto issue_qk = [&](int i, int st) {
+                const uint64_t qd = sdesc_sw128(smem_u32(sQ + i * C::Q_BYTES), 16, 1024);
+                const uint64_t kd = sdesc_sw128(smem_u32(sK + st * C::KV_BYTES), 16, 1024);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qa = smem_u32(sQ + i * C::Q_BYTES + (kk >> 2) * BM * 128 + (kk & 3) * 32);
-                    const uint32_t kb = smem_u32(sK + st * C::KV_BYTES + (kk >> 2) * BK * 128 + (kk & 3) * 32);
-                    umma_ss(tmem + C::S_COL(i), sdesc_sw128(qa, 16, 1024), sdesc_sw128(kb, 16, 1024), idesc_qk,
-                            kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss(tmem + C::S_COL(i), qd + (((kk >> 2) * BM * 128 + (kk & 3) * 32) >> 4),
+                            kd + (((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
             };
             auto issue_pv = [&](int i, int st, bool acc) {
+                const uint64_t vd = sdesc_sw128(smem_u32(sV + st * C::KV_BYTES), BK * 128, 1024);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {
-                    const uint32_t vb = smem_u32(sV + st * C::KV_BYTES + kk * 16 * 128);
-                    umma_ts(tmem + C::O_COL(i), tmem + C::S_COL(i) + kk * 8, sdesc_sw128(vb, BK * 128, 1024),
-                            idesc_pv, (acc || kk > 0) ? 1u : 0u);
-                }
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    umma_ts(tmem + C::O_COL(i), tmem + C::S_COL(i) + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
+                            (acc || kk > 0) ? 1u : 0u);
             };
             uint32_t kv_it = 0, q_it = 0, p_it[NQ] = {};
             bool ok = true;
