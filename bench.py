@@ -469,9 +469,11 @@ def measure_extras(torch, abi, A, W, dev, pk):
         ff = 4.0 * 0.5 * m["Hq"] * D * sum(L * L for L in lens)
         out = torch.empty_like(t["q"])
         lse = torch.empty((m["Hq"], m["total_q"]), dtype=torch.float32, device=dev)
+        fnb = abi.fa_varlen_fwd_workspace_size(16, m["total_q"], m["total_k"], 16, 16, D)
+        fws = torch.empty(fnb, dtype=torch.uint8, device=dev)    # the forward's dynamic schedule
         fms = timed(lambda: abi.fa_varlen_fwd(t["q"], t["k"], t["v"], out, lse, t["cu_q"], t["cu_k"], 16, m["max_q"],
-                                              m["max_k"], m["total_q"], m["total_k"], 16, 16, D, w.scale, 1, None, 0,
-                                              stream), 5)
+                                              m["max_k"], m["total_q"], m["total_k"], 16, 16, D, w.scale, 1, fws,
+                                              fnb, stream), 5)
         r = {"fwd_ms": fms, "fwd_tflops": ff / fms / 1e9, "total_tokens": m["total_q"]}
         dq, dk, dv = torch.empty_like(t["q"]), torch.empty_like(t["k"]), torch.empty_like(t["v"])
         nb = abi.fa_varlen_bwd_workspace_size(16, m["total_q"], m["total_k"], 16, 16, D)
@@ -596,9 +598,11 @@ def run_profile_case(args):
         lens = (t["cu_q"][1:] - t["cu_q"][:-1]).cpu().double()
         nbytes = 3.5 * float((4.0 * H * D * lens * lens * 0.5).sum())    # algorithmic FLOPs (fwd + bwd)
 
+        fws = torch.empty(256, dtype=torch.uint8, device=dev)    # the forward's dynamic schedule
+
         def fn():
             st = abi.fa_varlen_fwd(t["q"], t["k"], t["v"], out, lse, t["cu_q"], t["cu_k"], n, m["max_q"], m["max_k"],
-                                   T, T, H, H, D, w.scale, 1, None, 0, stream)
+                                   T, T, H, H, D, w.scale, 1, fws, 256, stream)
             return st | abi.fa_varlen_bwd(t["q"], t["k"], t["v"], out, t["do"], lse, dq, dk, dv, t["cu_q"], t["cu_k"],
                                           n, m["max_q"], m["max_k"], T, T, H, H, D, w.scale, 1, ws, nb, stream)
         name = f"varlen_16seq_L128-4096_H16_D{D}_causal_fwd+bwd"

@@ -58,7 +58,10 @@ def flash_attn_func(q, k, v, softmax_scale=None, causal=False, window_size=(-1, 
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
     out = torch.empty_like(q)
     lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=q.device)
-    _raise(abi.fa_fwd_ex(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, *_window(window_size)), "fa_fwd")
+    nb = abi.fa_fwd_workspace_size(B, Hq, Hkv, Sq, Sk, D)
+    ws = _workspace(nb, q.device)
+    _raise(abi.fa_fwd_ex(q, k, v, out, lse, B, Hq, Hkv, Sq, Sk, D, scale, causal, *_window(window_size), ws, nb),
+           "fa_fwd")
     return out, lse
 
 
@@ -92,8 +95,11 @@ def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, ma
     scale = 1.0 / math.sqrt(D) if softmax_scale is None else softmax_scale
     out = torch.empty_like(q)
     lse = torch.empty((Hq, total_q), dtype=torch.float32, device=q.device)
+    nb = abi.fa_varlen_fwd_workspace_size(nseq, total_q, total_k, Hq, Hkv, D)
+    ws = _workspace(nb, q.device)
     _raise(abi.fa_varlen_fwd_ex(q, k, v, out, lse, cu_seqlens_q, cu_seqlens_k, nseq, max_seqlen_q, max_seqlen_k,
-                                total_q, total_k, Hq, Hkv, D, scale, causal, *_window(window_size)), "fa_varlen_fwd")
+                                total_q, total_k, Hq, Hkv, D, scale, causal, *_window(window_size), ws, nb),
+           "fa_varlen_fwd")
     return out, lse
 
 

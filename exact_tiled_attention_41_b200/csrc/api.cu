@@ -157,7 +157,19 @@ int fa_get_device_status(fa_stream_t stream) {
 }
 
 // ----------------------------------------------------------------------- dense forward
-size_t fa_fwd_workspace_size(int, int, int, int, int, int) { return 0; }
+// The forward's workspace is optional: 256 bytes for the unit counter of its dynamic schedule.
+constexpr size_t kFwdWorkspace = 256;
+size_t fa_fwd_workspace_size(int, int, int, int, int, int) { return kFwdWorkspace; }
+
+// NULL: the static schedule (nothing to check); otherwise the counter, with the usual workspace rules.
+static int fwd_counter(void* workspace, size_t workspace_bytes, int** counter) {
+    *counter = nullptr;
+    if (workspace == nullptr) return FA_OK;
+    if (!aligned256(workspace)) return FA_ERR_ALIGNMENT;
+    if (workspace_bytes < kFwdWorkspace) return FA_ERR_WORKSPACE;
+    *counter = static_cast<int*>(workspace);
+    return FA_OK;
+}
 
 static int validate_dense(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int Sq, int Sk, int D,
                           float scale) {
@@ -205,16 +217,16 @@ int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, i
 int fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv, int Sq,
               int Sk, int D, float softmax_scale, int causal, int window_left, int window_right, void* workspace,
               size_t workspace_bytes, fa_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     int st = validate_dense(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale);
     if (st != FA_OK) return st;
     if (out == nullptr || lse == nullptr) return FA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+    int* counter = nullptr;
+    if ((st = fwd_counter(workspace, workspace_bytes, &counter)) != FA_OK) return st;
     Device dev;
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
     Problem pr = dense_problem(q, k, v, B, Hq, Hkv, Sq, Sk, D, softmax_scale, causal, window_left, window_right);
-    return launch_fwd(pr, out, lse, dev, static_cast<cudaStream_t>(stream));
+    return launch_fwd(pr, out, lse, counter, dev, static_cast<cudaStream_t>(stream));
 }
 
 // ----------------------------------------------------------------------- dense backward
@@ -291,7 +303,7 @@ static Problem varlen_problem(const void* q, const void* k, const void* v, const
     return pr;
 }
 
-size_t fa_varlen_fwd_workspace_size(int, int, int, int, int, int) { return 0; }
+size_t fa_varlen_fwd_workspace_size(int, int, int, int, int, int) { return kFwdWorkspace; }
 
 int fa_varlen_fwd(const void* q, const void* k, const void* v, void* out, float* lse, const int32_t* cu_seqlens_q,
                   const int32_t* cu_seqlens_k, int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q,
@@ -306,18 +318,18 @@ int fa_varlen_fwd_ex(const void* q, const void* k, const void* v, void* out, flo
                      const int32_t* cu_seqlens_k, int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q,
                      int total_k, int Hq, int Hkv, int D, float softmax_scale, int causal, int window_left,
                      int window_right, void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-    (void)workspace;
-    (void)workspace_bytes;
     int st = validate_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q, total_k,
                              Hq, Hkv, D, softmax_scale);
     if (st != FA_OK) return st;
     if (!out || !lse) return FA_ERR_INVALID_ARG;
     if (!aligned16(out) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+    int* counter = nullptr;
+    if ((st = fwd_counter(workspace, workspace_bytes, &counter)) != FA_OK) return st;
     Device dev;
     if (get_device(&dev) != FA_OK) return FA_ERR_CUDA;
     Problem pr = varlen_problem(q, k, v, cu_seqlens_q, cu_seqlens_k, num_seqs, max_seqlen_q, max_seqlen_k, total_q,
                                 total_k, Hq, Hkv, D, softmax_scale, causal, window_left, window_right);
-    return launch_fwd(pr, out, lse, dev, static_cast<cudaStream_t>(stream));
+    return launch_fwd(pr, out, lse, counter, dev, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_varlen_bwd_workspace_size(int num_seqs, int total_q, int total_k, int Hq, int Hkv, int D) {

@@ -45,7 +45,17 @@
 
 #include <math.h>
 
+#include <type_traits>
+
+#ifndef FA_BWD_FMA_EXP_EVERY
+#define FA_BWD_FMA_EXP_EVERY 6
+#endif
+
 namespace fa {
+
+// Share of the backward gradient step's exponentials computed on the FMA pipe (exp2_fma2): one pair
+// in kBwdFmaExpEvery, 0 = none.
+constexpr int kBwdFmaExpEvery = FA_BWD_FMA_EXP_EVERY;
 
 struct BwdParams {
     __nv_bfloat16* dk;
@@ -59,6 +69,8 @@ struct BwdParams {
     int n_blocks, num_units;
     float scale, scale_log2;
     int wl, wr;             // window sides, -1 = unbounded; a causal mask is wr = 0
+    int chunk;              // (sequence, KV head) groups per chunk of the unit list
+    int* counter;           // unit counter of the dynamic schedule (zeroed by the preprocess kernel)
     unsigned long long timeout_ns;
     int* status;
 };
@@ -68,11 +80,19 @@ struct BUnit {
     bool skip;
 };
 
+// Unit u: the list is cut into chunks of p.chunk (sequence, KV head) groups; inside a chunk the units
+// run key tile by key tile (the first tiles have the most work under a causal mask) over the chunk's
+// groups.  With p.chunk = all groups this is the plain heaviest-first order.
 __device__ __forceinline__ BUnit decode_bunit(const BwdParams& p, int u) {
     BUnit t;
-    const int per_n = p.num_seqs * p.Hkv;
-    const int n = u / per_n;          // key tile; the first tiles have the most work under a causal mask
-    const int r = u % per_n;
+    const int groups = p.num_seqs * p.Hkv;
+    const int per_chunk = p.chunk * p.n_blocks;
+    const int c = u / per_chunk;
+    const int g0 = c * p.chunk;
+    const int cs = min(p.chunk, groups - g0);
+    const int idx = u - c * per_chunk;
+    const int n = idx / cs;           // key tile
+    const int r = g0 + idx % cs;      // group
     t.b = r / p.Hkv;
     t.hk = r % p.Hkv;
     if (p.cu_q != nullptr) {
@@ -120,8 +140,8 @@ struct BwdCfg {
     static constexpr uint32_t OFF_K = 0, OFF_V = T_BYTES, OFF_Q = 2 * T_BYTES, OFF_DO = (2 + ST) * T_BYTES,
                               OFF_DS = (2 + 2 * ST) * T_BYTES, OFF_STAT = OFF_DS + DS_BYTES,
                               OFF_BAR = OFF_STAT + 2 * ST * 128 * 4;
-    static constexpr int NUM_BARS = 2 + 2 * ST + 9;
-    static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr int NUM_BARS = 2 + 2 * ST + 9 + 2 * kFeedSlots;
+    static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
     // tensor memory: dV | dK | S^T | dP^T.  After the gradient step the packed bf16 P^T and dS^T of each
     // 32-query half sit in that half's own 32 columns of S^T; dQ (fp32, D columns) is accumulated over
     // dP^T, whose values the warpgroups have read by then.
@@ -155,7 +175,9 @@ __global__ void __launch_bounds__(512, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* feed_slot = reinterpret_cast<int*>(tmem_slot + 4);
     const uint32_t b0 = smem_u32(bars);
+    const UnitFeed feed{feed_slot, b0 + 8u * (2 + 2 * ST + 9), b0 + 8u * (2 + 2 * ST + 9 + kFeedSlots)};
     // K and V of a unit arrive / are released separately: V is last read by the unit's last dP^T,
     // K by its last dQ (or S^T), so the next unit's V and first Q/dO tile load while those finish
     const uint32_t k_full = b0, k_free = b0 + 8;
@@ -189,6 +211,10 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bars + 2 + 2 * ST + 6, 128);  // p_full_hi: compute warpgroup 1 (query columns 64-127)
         mbar_init(bars + 2 + 2 * ST + 7, 1);    // v_full
         mbar_init(bars + 2 + 2 * ST + 8, 1);    // v_free
+        for (int s = 0; s < kFeedSlots; ++s) {
+            mbar_init(bars + 2 + 2 * ST + 9 + s, 1);                             // unit published
+            mbar_init(bars + 2 + 2 * ST + 9 + kFeedSlots + s, DQ ? 13 : 9);      // read by MMA, compute (, dQ) warps
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -215,8 +241,12 @@ __global__ void __launch_bounds__(512, 1)
             // -------------------------------------------------------- producer (whole warp)
             uint32_t unit_it = 0, q_it = 0;
             bool ok = true;
-            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-                if (u >= p.num_units) continue;
+            for (uint32_t fi = 0; ok; ++fi) {
+                int u = 0;
+                if (lane == 0 && !feed_put(feed, fi, p.counter, p.num_units, u, w)) u = -2;
+                u = __shfl_sync(0xffffffffu, u, 0);
+                if (u == -2) { ok = false; break; }
+                if (u < 0) break;
                 const BUnit t = decode_bunit(p, u);
                 if (t.skip || t.n_it == 0) continue;
                 // one query tile's Q and dO (TMA) and statistics (plain loads) into the next ring stage
@@ -282,8 +312,10 @@ __global__ void __launch_bounds__(512, 1)
                 constexpr uint32_t id_dq = idesc_bf16_f32(128, D, true, true);       // dQ, all D columns
                 uint32_t unit_it = 0, q_it = 0, g_it = 0;
                 bool ok = true;
-                for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-                    if (u >= p.num_units) continue;
+                for (uint32_t fi = 0; ok; ++fi) {
+                    int u;
+                    if (!feed_get(feed, fi, u, w, false)) { ok = false; break; }
+                    if (u < 0) break;
                     const BUnit t = decode_bunit(p, u);
                     if (t.skip || t.n_it == 0) continue;
                     if (!mbar_wait(k_full, unit_it & 1, w)) { ok = false; break; }
@@ -365,8 +397,10 @@ __global__ void __launch_bounds__(512, 1)
         const uint32_t lb = tmem_lane_base(wq);
         uint32_t g_it = 0;
         bool ok = true;
-        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-            if (u >= p.num_units) continue;
+        for (uint32_t fi = 0; ok; ++fi) {
+            int u;
+            if (!feed_get(feed, fi, u, w, true)) { ok = false; break; }
+            if (u < 0) break;
             const BUnit t = decode_bunit(p, u);
             if (t.skip || t.n_it == 0) continue;
             for (int it = 0; it < t.n_it; ++it, ++g_it) {
@@ -408,8 +442,10 @@ __global__ void __launch_bounds__(512, 1)
         const float c2 = p.scale_log2;
         uint32_t unit_it = 0, q_it = 0, g_it = 0;
         bool ok = true;
-        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-            if (u >= p.num_units) continue;
+        for (uint32_t fi = 0; ok; ++fi) {
+            int u;
+            if (!feed_get(feed, fi, u, w, true)) { ok = false; break; }
+            if (u < 0) break;
             const BUnit t = decode_bunit(p, u);
             if (t.skip) continue;
             const int kj = t.n0 + r;                 // key index inside the sequence
@@ -449,7 +485,14 @@ __global__ void __launch_bounds__(512, 1)
                 const float* del_t = sDel + st * 128 + 64 * gq;
                 const float2 c2v = make_float2(c2, c2);
                 uint8_t* ds_row = smem + C::OFF_DS + gq * 128 * 128 + r * 128;
-                // the two 32-column halves one after the other, so only one half's values are live
+                // the two 32-column halves one after the other, so only one half's values are live;
+                // on tiles without masking or rows past the sequence one pair in kBwdFmaExpEvery takes
+                // its exponentials from the FMA pipe (both warpgroups run this step at the same time, so
+                // they share the exp2 unit; one pair in 6 measured best: +3 % dense, +6 % long-context
+                // GQA, +7 % varlen D = 64 over none, ahead of one in 3 or 4)
+                auto grad = [&](auto poly) {
+                constexpr int kEvery = decltype(poly)::value ? kBwdFmaExpEvery : 0;
+                constexpr int kMod = kEvery > 0 ? kEvery : 1;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t sh[32], dh[32];
@@ -469,7 +512,8 @@ __global__ void __launch_bounds__(512, 1)
                             const float2 sv = make_float2(__uint_as_float(sh[e + x]), __uint_as_float(sh[e + x + 1]));
                             const float2 dv = make_float2(__uint_as_float(dh[e + x]), __uint_as_float(dh[e + x + 1]));
                             const float2 a = ffma2(sv, c2v, make_float2(la, lbv));
-                            float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                            float2 pr = (kEvery > 0 && ((e + x) / 2) % kMod == kMod - 1)
+                                            ? exp2_fma2(a) : make_float2(ex2_approx(a.x), ex2_approx(a.y));
                             if (any_mask) {
                                 const int qc = 64 * gq + half * 32 + e + x;
                                 pr.x = (qc >= qmin && qc <= qmax) ? pr.x : 0.f;
@@ -491,6 +535,9 @@ __global__ void __launch_bounds__(512, 1)
                             make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
                     }
                 }
+                };
+                if (kBwdFmaExpEvery > 0 && !any_mask && m0 + 128 <= t.Lq) grad(std::true_type{});
+                else grad(std::false_type{});
                 tmem_st_wait();
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -859,6 +906,12 @@ __global__ void __launch_bounds__(384, 1)
                     const bool any_mask = __any_sync(0xffffffffu, !(qmin <= 0 && qmax >= 63));
                     const float* lse_t = sLSE + st * 64;
                     const float* del_t = sDel + st * 64;
+                    // the same FMA-pipe share of the exponentials as bwd_kernel, on the same elements and under
+                    // the same condition (no masked column in the warp's 64, the whole 128-row query tile inside
+                    // the sequence), so both backward modes compute identical P^T and dS^T
+                    auto grad = [&](auto poly) {
+                    constexpr int kEvery = decltype(poly)::value ? kBwdFmaExpEvery : 0;
+                    constexpr int kMod = kEvery > 0 ? kEvery : 1;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         uint32_t sh[32], dh[32];
@@ -878,7 +931,8 @@ __global__ void __launch_bounds__(384, 1)
                                 const float2 sv = make_float2(__uint_as_float(sh[e + x]), __uint_as_float(sh[e + x + 1]));
                                 const float2 dv = make_float2(__uint_as_float(dh[e + x]), __uint_as_float(dh[e + x + 1]));
                                 const float2 a = ffma2(sv, c2v, make_float2(la, lbv));
-                                float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                                float2 pr = (kEvery > 0 && ((e + x) / 2) % kMod == kMod - 1)
+                                                ? exp2_fma2(a) : make_float2(ex2_approx(a.x), ex2_approx(a.y));
                                 if (any_mask) {
                                     const int qc = half * 32 + e + x;
                                     pr.x = (qc >= qmin && qc <= qmax) ? pr.x : 0.f;
@@ -893,6 +947,9 @@ __global__ void __launch_bounds__(384, 1)
                         tmem_st16(tmem + lb + C::COL_S(gb) + 32 * half, pp);
                         tmem_st16(tmem + lb + C::COL_S(gb) + 32 * half + 16, dd);
                     }
+                    };
+                    if (kBwdFmaExpEvery > 0 && !any_mask && row0 - 64 * qh + 128 <= t.Lq) grad(std::true_type{});
+                    else grad(std::false_type{});
                     tmem_st_wait();
                     tc_fence_before();
                     mbar_arrive(p_full(gb));
@@ -945,14 +1002,16 @@ __global__ void __launch_bounds__(384, 1)
 
 // ---------------------------------------------------------------------------- preprocess
 // One warp per (query token, head): Delta = sum_d dO * O (fp32), LSE2 = LSE * log2(e)
-// (+inf where LSE = -inf).  Also zeroes the dQ accumulator (grid-stride) unless dq_acc is NULL.
+// (+inf where LSE = -inf).  Also zeroes the dQ accumulator (grid-stride) unless dq_acc is NULL, and
+// the main kernel's unit counter unless counter is NULL.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
                                                       const float* lse, float* lse2, float* delta, float* dq_acc,
-                                                      int Tq, int Hq, int Sq, long long lse_sB, long long lse_sH,
-                                                      int lse_sT) {
+                                                      int* counter, int Tq, int Hq, int Sq, long long lse_sB,
+                                                      long long lse_sH, int lse_sT) {
     const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
+    if (counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *counter = 0;
     const long long rows = static_cast<long long>(Tq) * Hq;
     if (dq_acc != nullptr) {
         const long long n4 = rows * D / 4;
@@ -1028,11 +1087,35 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(const float* dq_acc, _
     }
 }
 
+// fp32 dQ accumulator | LSE2 | Delta | 256 bytes for the main kernel's unit counter
 size_t bwd_workspace_bytes(long long Tq, int Hq, int D) {
     const size_t acc = static_cast<size_t>(Tq) * Hq * D * 4;
     const size_t stat = static_cast<size_t>(Tq) * Hq * 4;
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-    return up(acc) + 2 * up(stat);
+    return up(acc) + 2 * up(stat) + 256;
+}
+
+int* bwd_unit_counter(void* workspace, long long Tq, int Hq, int D) {
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t acc = static_cast<size_t>(Tq) * Hq * D * 4;
+    const size_t stat = static_cast<size_t>(Tq) * Hq * 4;
+    return reinterpret_cast<int*>(static_cast<char*>(workspace) + up(acc) + 2 * up(stat));
+}
+
+// Key-tile units are dealt in chunks of `chunk` (sequence, KV head) groups, heaviest key tile first
+// inside a chunk, so that the CTAs working at one time share the Q, dO and dQ accumulator of a few
+// heads in L2.  A chunk holds enough units for every CTA (twice over) and, beyond that, as many groups
+// as fit about 96 MB of Q, dO and fp32 dQ.
+int bwd_chunk_groups(int num_groups, int units_per_group, int group_q_heads, int max_len, int D, int num_sms) {
+    const double per_group = static_cast<double>(group_q_heads) * max_len * D * 8.0;
+    long long by_l2 = static_cast<long long>(96.0 * (1 << 20) / (per_group > 1.0 ? per_group : 1.0));
+    const long long by_balance = (2LL * num_sms + units_per_group - 1) / (units_per_group > 0 ? units_per_group : 1);
+    long long c = by_l2 > by_balance ? by_l2 : by_balance;
+    if (c < 1) c = 1;
+    if (c > num_groups) c = num_groups;
+    // chunks of equal size, so the schedule does not end on a lone small chunk
+    const long long n_chunks = (num_groups + c - 1) / c;
+    return static_cast<int>((num_groups + n_chunks - 1) / n_chunks);
 }
 
 template <int D, bool DQ>
@@ -1051,7 +1134,8 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
         if (blocks > cap) blocks = cap;
         bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
-            DQ ? dq_acc : nullptr, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+            DQ ? dq_acc : nullptr, bwd_unit_counter(workspace, pr.Tq, pr.Hq, D), pr.Tq, pr.Hq, pr.Sq, pr.lse_sB,
+            pr.lse_sH, pr.lse_sT);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
 
@@ -1089,6 +1173,8 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     p.scale_log2 = pr.scale * 1.4426950408889634f;
     p.wl = pr.wl;
     p.wr = pr.wr;
+    p.chunk = bwd_chunk_groups(pr.num_seqs * pr.Hkv, p.n_blocks, p.group, pr.Sq, D, dev.num_sms);
+    p.counter = bwd_unit_counter(workspace, pr.Tq, pr.Hq, D);
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
 
@@ -1132,7 +1218,7 @@ static int run_bwd_pp(const Problem& pr, const void* out, const void* dout, cons
         if (blocks > cap) blocks = cap;
         bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
-            nullptr, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+            nullptr, nullptr, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
     alignas(64) CUtensorMap mq, mk, mv, mdo;
@@ -1166,6 +1252,8 @@ static int run_bwd_pp(const Problem& pr, const void* out, const void* dout, cons
     p.scale_log2 = pr.scale * 1.4426950408889634f;
     p.wl = pr.wl;
     p.wr = pr.wr;
+    p.chunk = pr.num_seqs * pr.Hkv;   // the static heaviest-first order over all groups
+    p.counter = nullptr;
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
 
@@ -1204,7 +1292,8 @@ static int run_bwd256(const Problem& pr, const void* out, const void* dout, cons
     if (blocks > cap) blocks = cap;
     bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
-        det ? nullptr : dq_acc, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+        det ? nullptr : dq_acc, bwd_unit_counter(workspace, pr.Tq, pr.Hq, D), pr.Tq, pr.Hq, pr.Sq, pr.lse_sB,
+        pr.lse_sH, pr.lse_sT);
     if (cudaPeekAtLastError() != cudaSuccess) return 5;
     const int st = launch_bwd256_main(pr, dout, lse2, delta, dq_acc, dq, dk, dv, !det, dev, stream);
     if (st != 0 || !det) return st;

@@ -40,6 +40,8 @@ struct B256Params {
     int num_units;
     float scale, scale_log2;
     int wl, wr;             // window sides, -1 = unbounded; a causal mask is wr = 0
+    int n_blocks, chunk;    // key tiles per sequence; (sequence, KV head) groups per chunk of the unit list
+    int* counter;           // unit counter of the dynamic schedule (zeroed by the preprocess kernel)
     unsigned long long timeout_ns;
     int* status;
 };
@@ -49,13 +51,20 @@ struct U256 {
     bool skip;
 };
 
+// Unit u: chunks of p.chunk (sequence, KV head) groups; inside a chunk, key tile by key tile (the
+// first tiles have the most work under a causal mask) over the chunk's groups and both head-dim halves.
 __device__ __forceinline__ U256 decode_u256(const B256Params& p, int u) {
     U256 t;
-    const int per_n = p.num_seqs * p.Hkv * 2;
-    const int n = u / per_n;            // key tile; the first tiles have the most work under a causal mask
-    int r = u % per_n;
-    t.hh = r & 1;                       // the two halves of a key tile run on neighbouring CTAs
-    r >>= 1;
+    const int groups = p.num_seqs * p.Hkv;
+    const int per_chunk = p.chunk * p.n_blocks * 2;
+    const int c = u / per_chunk;
+    const int g0 = c * p.chunk;
+    const int cs = min(p.chunk, groups - g0);
+    const int idx = u - c * per_chunk;
+    const int n = idx / (2 * cs);       // key tile
+    int r = idx % (2 * cs);
+    t.hh = r & 1;                       // the two halves of a key tile are taken one after the other
+    r = g0 + (r >> 1);
     t.b = r / p.Hkv;
     t.hk = r % p.Hkv;
     if (p.cu_q != nullptr) {
@@ -94,8 +103,8 @@ struct Cfg {
     static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_Q = 2 * KV_BYTES, OFF_DO = OFF_Q + QT_BYTES,
                               OFF_DS = OFF_DO + QT_BYTES,               // dS^T [128 keys][64 queries], 16 KB
                               OFF_STAT = OFF_DS + 128 * 128, OFF_BAR = OFF_STAT + 2 * 64 * 4;
-    static constexpr int NUM_BARS = 9;
-    static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr int NUM_BARS = 9 + 2 * kFeedSlots;
+    static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
     static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
     static constexpr int THREADS = 384, LAUNCH_REGS = 168, COMPUTE_REGS = 232, OTHER_REGS = 136;
     static_assert(128 * COMPUTE_REGS + 2 * 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
@@ -113,7 +122,9 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* feed_slot = reinterpret_cast<int*>(tmem_slot + 4);
     const uint32_t b0 = smem_u32(bars);
+    const UnitFeed feed{feed_slot, b0 + 8u * 9, b0 + 8u * (9 + kFeedSlots)};
     const uint32_t kv_full = b0, kv_empty = b0 + 8, q_full = b0 + 16, q_empty = b0 + 24, s_full = b0 + 32,
                    p_full = b0 + 40, dq_full = b0 + 48, dq_empty = b0 + 56, dkv_full = b0 + 64;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -133,6 +144,10 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(bars + 6, 1);
         mbar_init(bars + 7, 128);    // dq_empty
         mbar_init(bars + 8, 1);
+        for (int s = 0; s < kFeedSlots; ++s) {
+            mbar_init(bars + 9 + s, 1);                              // unit published
+            mbar_init(bars + 9 + kFeedSlots + s, DQ ? 9 : 5);        // read by MMA, compute (, dQ) warps
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -158,8 +173,12 @@ __global__ void __launch_bounds__(384, 1)
         if (warp == PRODUCER) {
             uint32_t unit_it = 0, q_it = 0;
             bool ok = true;
-            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-                if (u >= p.num_units) continue;
+            for (uint32_t fi = 0; ok; ++fi) {
+                int u = 0;
+                if (lane == 0 && !feed_put(feed, fi, p.counter, p.num_units, u, w)) u = -2;
+                u = __shfl_sync(0xffffffffu, u, 0);
+                if (u == -2) { ok = false; break; }
+                if (u < 0) break;
                 const U256 t = decode_u256(p, u);
                 if (t.skip || t.n_it == 0) continue;
                 if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
@@ -209,8 +228,10 @@ __global__ void __launch_bounds__(384, 1)
                 constexpr uint32_t id_q = idesc_bf16_f32(128, 64, true, true);       // dQ^T half
                 uint32_t unit_it = 0, q_it = 0;
                 bool ok = true;
-                for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-                    if (u >= p.num_units) continue;
+                for (uint32_t fi = 0; ok; ++fi) {
+                    int u;
+                    if (!feed_get(feed, fi, u, w, false)) { ok = false; break; }
+                    if (u < 0) break;
                     const U256 t = decode_u256(p, u);
                     if (t.skip || t.n_it == 0) continue;
                     if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
@@ -276,8 +297,10 @@ __global__ void __launch_bounds__(384, 1)
             const uint32_t lb = tmem_lane_base(wq);
             uint32_t q_it = 0;
             bool ok = true;
-            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-                if (u >= p.num_units) continue;
+            for (uint32_t fi = 0; ok; ++fi) {
+                int u;
+                if (!feed_get(feed, fi, u, w, true)) { ok = false; break; }
+                if (u < 0) break;
                 const U256 t = decode_u256(p, u);
                 if (t.skip || t.n_it == 0) continue;
                 for (int it = 0; it < t.n_it; ++it, ++q_it) {
@@ -311,8 +334,10 @@ __global__ void __launch_bounds__(384, 1)
         const float c2 = p.scale_log2;
         uint32_t unit_it = 0, q_it = 0;
         bool ok = true;
-        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
-            if (u >= p.num_units) continue;
+        for (uint32_t fi = 0; ok; ++fi) {
+            int u;
+            if (!feed_get(feed, fi, u, w, true)) { ok = false; break; }
+            if (u < 0) break;
             const U256 t = decode_u256(p, u);
             if (t.skip) continue;
             const int kj = t.n0 + r;
@@ -478,6 +503,9 @@ static int run_bwd256(const Problem& pr, const void* dout, const float* lse2, co
     p.scale_log2 = pr.scale * 1.4426950408889634f;
     p.wl = pr.wl;
     p.wr = pr.wr;
+    p.n_blocks = (pr.Sk + 127) / 128;
+    p.chunk = bwd_chunk_groups(pr.num_seqs * pr.Hkv, 2 * p.n_blocks, p.group, pr.Sq, D, dev.num_sms);
+    p.counter = bwd_unit_counter(dq_acc, pr.Tq, pr.Hq, D);   // dq_acc is the start of the workspace
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
     auto kern = bwd256_kernel<DQ>;

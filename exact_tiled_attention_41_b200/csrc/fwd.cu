@@ -21,8 +21,11 @@
 //   Order per KV tile j: PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1), so the tensor
 //   core computes one tile's scores while the other tile's softmax runs.
 //   * work units (sequence, head, block of NQ*128 query rows) are listed
-//     heaviest first (query blocks with most KV tiles first for causal masks)
-//     and dealt to the persistent CTAs in boustrophedon order (snake_unit);
+//     heaviest first (query blocks with most KV tiles first for causal masks),
+//     in chunks of heads whose K and V fit L2 together; with a workspace the
+//     CTAs take them from a counter as they finish (dynamic), without one they
+//     are dealt in boustrophedon order (snake_unit); the producer publishes each
+//     unit to the other roles through a small shared-memory ring;
 //     each query tile only visits the KV tiles its mask can reach: causal
 //     blocks stop at the last KV tile they can see, and a sliding window
 //     (README, flash_attn_func docstring: query i keeps the keys in
@@ -55,6 +58,8 @@ struct FwdParams {
     int wl, wr;   // window sides, -1 = unbounded; a causal mask is wr = 0
     long long lse_sB, lse_sH;
     int lse_sT;
+    int chunk;      // (sequence, query head) groups per chunk of the unit list
+    int* counter;   // unit counter of the dynamic schedule (zeroed before the launch), or NULL: static
     unsigned long long timeout_ns;
     int* status;
 };
@@ -70,12 +75,20 @@ struct Unit {
 
 // LOCAL: the window has a bounded left side, so query tiles may start past KV tile 0.
 // Without it kv0 and lo[] are 0 and the accessors below fold them away.
+// Unit u: the list is cut into chunks of p.chunk (sequence, query head) groups; inside a chunk the units
+// run query block by query block, the blocks that see the most keys first, over the chunk's groups (so
+// the CTAs of one moment share a few heads' K and V in L2).  p.chunk = all groups: heaviest first.
 template <int ROWS, int BK, bool LOCAL>
 __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
     Unit t;
-    const int per_m = p.num_seqs * p.Hq;
-    const int m = p.m_blocks - 1 - u / per_m;
-    const int r = u % per_m;
+    const int groups = p.num_seqs * p.Hq;
+    const int per_chunk = p.chunk * p.m_blocks;
+    const int c = u / per_chunk;
+    const int g0 = c * p.chunk;
+    const int cs = min(p.chunk, groups - g0);
+    const int idx = u - c * per_chunk;
+    const int m = p.m_blocks - 1 - idx / cs;
+    const int r = g0 + idx % cs;
     t.b = r / p.Hq;
     t.h = r % p.Hq;
     if (p.cu_q != nullptr) {
@@ -163,8 +176,8 @@ struct FwdCfg {
     static constexpr int NCHUNK = D / 64;
     static constexpr uint32_t Q_BYTES = BM * D * 2;
     static constexpr uint32_t KV_BYTES = BK * D * 2;
-    static constexpr int NUM_BARS = 5 * NQ + 4 * KST;
-    static constexpr size_t SMEM = 1024 + NQ * Q_BYTES + 2 * KST * KV_BYTES + NUM_BARS * 8 + 16;
+    static constexpr int NUM_BARS = 5 * NQ + 4 * KST + 2 * kFeedSlots;
+    static constexpr size_t SMEM = 1024 + NQ * Q_BYTES + 2 * KST * KV_BYTES + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
     // NQ softmax warpgroups + one warpgroup holding the producer warp, the MMA warp and two idle warps
     static constexpr int THREADS = (4 * NQ + 4) * 32;
     // register split with setmaxnreg (NQ = 2): launch at 168 per thread (384 x 168 = 64512),
@@ -199,7 +212,10 @@ __host__ __device__ constexpr int fma_exp_every(int D) {
 }
 constexpr float kLn2 = 0.69314718055994530942f;
 
-template <int D, int NQ, int BK, int KST, bool LOCAL>
+// DYN: units come from p.counter through the shared-memory feed (varlen batches, head chunks sized for
+// L2); otherwise each role walks the static boustrophedon deal itself (dense problems whose K and V fit
+// L2: the static deal is balanced there, and the feed's per-unit hand-off measured 2-3 % slower).
+template <int D, int NQ, int BK, int KST, bool LOCAL, bool DYN>
 __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ FwdParams p) {
@@ -215,8 +231,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(sV + KST * C::KV_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* feed_slot = reinterpret_cast<int*>(tmem_slot + 4);
 
     const uint32_t bar0 = smem_u32(bars);
+    const UnitFeed feed{feed_slot, bar0 + 8u * (5 * NQ + 4 * KST), bar0 + 8u * (5 * NQ + 4 * KST + kFeedSlots)};
     auto q_full = [&](int i) { return bar0 + 8u * (0 * NQ + i); };
     auto q_empty = [&](int i) { return bar0 + 8u * (1 * NQ + i); };
     auto s_full = [&](int i) { return bar0 + 8u * (2 * NQ + i); };
@@ -241,6 +259,10 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             mbar_init(bars + 4 * NQ + i, 1);
         }
         for (int s = 0; s < 4 * KST; ++s) mbar_init(bars + 5 * NQ + s, 1);
+        for (int s = 0; s < kFeedSlots; ++s) {
+            mbar_init(bars + 5 * NQ + 4 * KST + s, 1);                       // unit published
+            mbar_init(bars + 5 * NQ + 4 * KST + kFeedSlots + s, 1 + 4 * NQ); // read by the MMA and softmax warps
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -265,12 +287,35 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     if (warp == PRODUCER) {
         if (lane == 0) {
             uint32_t kv_it = 0, q_it = 0;
-            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0; u = snake_unit(++k, p.num_units)) {
+            // DYN: units come from the counter; the next one is taken and published one ahead of the one
+            // being loaded, so the counter's latency is hidden.  Static: the boustrophedon deal.
+            int k_static = 0;
+            auto take = [&]() -> int {
+                if constexpr (DYN) {
+                    const int v = atomicAdd(p.counter, 1);
+                    return v < p.num_units ? v : -1;
+                } else {
+                    return snake_unit(k_static++, p.num_units);   // -1 at the end, num_units = an empty slot
+                }
+            };
+            auto publish = [&](uint32_t it, int v) -> bool {
+                if constexpr (!DYN) return true;
+                const uint32_t s = it % kFeedSlots;
+                if (it >= kFeedSlots && !mbar_wait(feed.empty0 + 8 * s, ((it / kFeedSlots) - 1) & 1, w)) return false;
+                feed.slot[s] = v;
+                mbar_arrive(feed.full0 + 8 * s);
+                return true;
+            };
+            int u_next = take();
+            bool ok = publish(0, u_next);
+            for (uint32_t fi = 0; ok && u_next >= 0; ++fi) {
+                const int u = u_next;
+                u_next = take();
+                if (!publish(fi + 1, u_next)) break;
                 if (u >= p.num_units) continue;
                 const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
                 if (t.skip || t.n_kv == 0) continue;
                 const int hk = t.h / p.group;
-                bool ok = true;
                 for (int i = 0; i < NQ && ok; ++i) {
                     if (q_it > 0 && !mbar_wait(q_empty(i), (q_it - 1) & 1, w)) ok = false;
                     if (!ok) break;
@@ -326,7 +371,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             };
             uint32_t kv_it = 0, q_it = 0, p_it[NQ] = {};
             bool ok = true;
-            for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+            for (uint32_t fi = 0; ok; ++fi) {
+                int u;
+                if constexpr (DYN) {
+                    if (!feed_get(feed, fi, u, w, false)) break;
+                } else {
+                    u = snake_unit(static_cast<int>(fi), p.num_units);
+                }
+                if (u < 0) break;
                 if (u >= p.num_units) continue;
                 const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
                 if (t.skip || t.n_kv == 0) continue;
@@ -403,7 +455,14 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
         const float c2 = p.scale_log2;
         uint32_t s_it = 0, pv_total = 0;
         bool ok = true;
-        for (int k = 0, u = snake_unit(0, p.num_units); u >= 0 && ok; u = snake_unit(++k, p.num_units)) {
+        for (uint32_t fi = 0; ok; ++fi) {
+            int u;
+            if constexpr (DYN) {
+                if (!feed_get(feed, fi, u, w, true)) break;
+            } else {
+                u = snake_unit(static_cast<int>(fi), p.num_units);
+            }
+            if (u < 0) break;
             if (u >= p.num_units) continue;
             const Unit t = decode_unit<ROWS, BK, LOCAL>(p, u);
             if (t.skip) continue;
@@ -561,8 +620,23 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
     }
 }
 
-template <int D, int NQ, int BK, int KST, bool LOCAL>
-static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream) {
+// Groups (sequence, query head) per chunk of the unit list: every group of a chunk keeps its K and V
+// (shared by the group of query heads reading one KV head) in L2 while the chunk's query blocks run;
+// chunks of about 96 MB of K and V, and at least twice as many units as CTAs.
+static int fwd_chunk_groups(const Problem& pr, int D, int m_blocks, int num_sms) {
+    const int groups = pr.num_seqs * pr.Hq;
+    const double kv_per_group = 4.0 * pr.Sk * D / (pr.Hq / pr.Hkv);
+    long long c = static_cast<long long>(96.0 * (1 << 20) / (kv_per_group > 1.0 ? kv_per_group : 1.0));
+    const long long by_balance = (2LL * num_sms + m_blocks - 1) / m_blocks;
+    if (c < by_balance) c = by_balance;
+    if (c < 1) c = 1;
+    if (c > groups) c = groups;
+    const long long n_chunks = (groups + c - 1) / c;
+    return static_cast<int>((groups + n_chunks - 1) / n_chunks);
+}
+
+template <int D, int NQ, int BK, int KST, bool LOCAL, bool DYN>
+static int run_fwd(const Problem& pr, void* out, float* lse, int* counter, const Device& dev, cudaStream_t stream) {
     using C = FwdCfg<D, NQ, BK, KST>;
     alignas(64) CUtensorMap mq, mk, mv;
     const uint64_t rq = static_cast<uint64_t>(pr.Hq) * D * 2, rk = static_cast<uint64_t>(pr.Hkv) * D * 2;
@@ -593,11 +667,16 @@ static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, 
     p.lse_sB = pr.lse_sB;
     p.lse_sH = pr.lse_sH;
     p.lse_sT = pr.lse_sT;
+    // DYN (a counter from the caller's workspace): head-chunked order taken dynamically; otherwise the
+    // static heaviest-first deal over all groups
+    p.counter = DYN ? counter : nullptr;
+    p.chunk = DYN ? fwd_chunk_groups(pr, D, p.m_blocks, dev.num_sms) : pr.num_seqs * pr.Hq;
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
     if (p.num_units == 0) return 0;
+    if (DYN && cudaMemsetAsync(counter, 0, sizeof(int), stream) != cudaSuccess) return 5;
 
-    auto kern = fwd_kernel<D, NQ, BK, KST, LOCAL>;
+    auto kern = fwd_kernel<D, NQ, BK, KST, LOCAL, DYN>;
     static bool attr_set[64] = {};
     if (!attr_set[dev.id & 63]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(C::SMEM)) !=
@@ -618,15 +697,26 @@ static int run_fwd(const Problem& pr, void* out, float* lse, const Device& dev, 
     return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
 }
 
-int launch_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream) {
+template <int D, int NQ, int BK, int KST>
+static int run_fwd_d(const Problem& pr, void* out, float* lse, int* counter, const Device& dev,
+                     cudaStream_t stream) {
+    // the dynamic schedule where it pays: varlen batches (unequal lengths unbalance the static deal) and
+    // problems whose K and V do not fit L2 together (head chunks); it needs the caller's workspace
+    const int m_blocks = (pr.Sq + 128 * NQ - 1) / (128 * NQ);
+    const bool dyn = counter != nullptr &&
+                     (pr.cu_q != nullptr || fwd_chunk_groups(pr, D, m_blocks, dev.num_sms) < pr.num_seqs * pr.Hq);
     const bool local = pr.wl >= 0;
+    if (dyn) return local ? run_fwd<D, NQ, BK, KST, true, true>(pr, out, lse, counter, dev, stream)
+                          : run_fwd<D, NQ, BK, KST, false, true>(pr, out, lse, counter, dev, stream);
+    return local ? run_fwd<D, NQ, BK, KST, true, false>(pr, out, lse, nullptr, dev, stream)
+                 : run_fwd<D, NQ, BK, KST, false, false>(pr, out, lse, nullptr, dev, stream);
+}
+
+int launch_fwd(const Problem& pr, void* out, float* lse, int* counter, const Device& dev, cudaStream_t stream) {
     switch (pr.D) {
-        case 64: return local ? run_fwd<64, 2, 128, 4, true>(pr, out, lse, dev, stream)
-                              : run_fwd<64, 2, 128, 4, false>(pr, out, lse, dev, stream);
-        case 128: return local ? run_fwd<128, 2, 128, 2, true>(pr, out, lse, dev, stream)
-                               : run_fwd<128, 2, 128, 2, false>(pr, out, lse, dev, stream);
-        case 256: return local ? run_fwd<256, 1, 128, 1, true>(pr, out, lse, dev, stream)
-                               : run_fwd<256, 1, 128, 1, false>(pr, out, lse, dev, stream);
+        case 64: return run_fwd_d<64, 2, 128, 4>(pr, out, lse, counter, dev, stream);
+        case 128: return run_fwd_d<128, 2, 128, 2>(pr, out, lse, counter, dev, stream);
+        case 256: return run_fwd_d<256, 1, 128, 1>(pr, out, lse, counter, dev, stream);
         default: return 2;
     }
 }

@@ -44,9 +44,11 @@ int get_device(Device* dev);     // fills for the current device; returns FA sta
 void prof_before(int kernel_id, cudaStream_t s);
 void prof_after(int kernel_id, cudaStream_t s);
 
-int launch_fwd(const Problem& pr, void* out, float* lse, const Device& dev, cudaStream_t stream);
+int launch_fwd(const Problem& pr, void* out, float* lse, int* counter, const Device& dev, cudaStream_t stream);
 
 size_t bwd_workspace_bytes(long long Tq, int Hq, int D);
+int* bwd_unit_counter(void* workspace, long long Tq, int Hq, int D);
+int bwd_chunk_groups(int num_groups, int units_per_group, int group_q_heads, int max_len, int D, int num_sms);
 // head dim 256: main backward kernel + dQ convert (after the shared preprocess); with_dq = false
 // leaves dq alone (the deterministic backward computes it with launch_bwd_dq)
 int launch_bwd256_main(const Problem& pr, const void* dout, const float* lse2, const float* delta, float* dq_acc,

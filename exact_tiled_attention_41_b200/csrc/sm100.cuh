@@ -370,6 +370,42 @@ __device__ __forceinline__ void stg_flush(const uint8_t* stg, uint8_t* dst, long
 
 __device__ __forceinline__ int elect_lane0() { return (threadIdx.x & 31) == 0; }
 
+// Dynamic persistent schedule: one thread of the producer warp takes unit indices from a global
+// counter (zeroed before the launch, on the same stream) and hands them to the CTA's other roles
+// through kFeedSlots shared-memory slots.  Slot s has a full barrier (one arrival: the producer,
+// whose arrive releases the slot write) and an empty barrier (one arrival per consuming warp).
+// When the list is exhausted the producer publishes -1, and every role stops there.
+constexpr int kFeedSlots = 4;
+
+struct UnitFeed {
+    int* slot;         // [kFeedSlots] in shared memory
+    uint32_t full0;    // full barrier of slot s: full0 + 8 s
+    uint32_t empty0;   // empty barrier of slot s: empty0 + 8 s
+};
+
+// Producer thread: publish this CTA's it-th unit (or -1); false = gave up waiting for the slot.
+__device__ __forceinline__ bool feed_put(const UnitFeed& f, uint32_t it, int* counter, int num_units, int& u,
+                                         const Watch& w) {
+    const uint32_t s = it % kFeedSlots;
+    if (it >= kFeedSlots && !mbar_wait(f.empty0 + 8 * s, ((it / kFeedSlots) - 1) & 1, w)) return false;
+    const int v = atomicAdd(counter, 1);
+    u = v < num_units ? v : -1;
+    f.slot[s] = u;
+    mbar_arrive(f.full0 + 8 * s);
+    return true;
+}
+
+// Consumer: the it-th unit (every calling thread waits; lane 0 of each warp releases the slot, so the
+// whole warp must call it together, or only lane 0 when the warp's other lanes never consume).
+__device__ __forceinline__ bool feed_get(const UnitFeed& f, uint32_t it, int& u, const Watch& w, bool whole_warp) {
+    const uint32_t s = it % kFeedSlots;
+    if (!mbar_wait(f.full0 + 8 * s, (it / kFeedSlots) & 1, w)) return false;
+    u = f.slot[s];
+    if (whole_warp) __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(f.empty0 + 8 * s);
+    return true;
+}
+
 // Persistent schedule over work units sorted heaviest first: round k of CTA c takes unit
 // k*G + c on even rounds and k*G + (G-1-c) on odd rounds (a boustrophedon), so the CTA that
 // got the heaviest unit of one round gets the lightest of the next.  Returns -1 past the end

@@ -76,7 +76,13 @@ enum fa_status {
  *   q    [B, Sq, Hq,  D]      k, v [B, Sk, Hkv, D]      out [B, Sq, Hq, D]
  *   lse  [B, Hq, Sq] float32 (required: the backward consumes it)
  * Source: README, "How to use FlashAttention" (definition) and the
- * flash_attn_func docstring (shapes, GQA, causal).  Workspace: none.
+ * flash_attn_func docstring (shapes, GQA, causal).
+ * Workspace: optional.  With fa_fwd_workspace_size() bytes (256) the persistent
+ * kernel takes its work units from a counter there as CTAs finish (balanced on
+ * unequal sequence lengths; heads grouped so their K and V stay in L2), zeroed
+ * on `stream` by the call itself; with workspace = NULL the units are dealt
+ * statically.  The result does not depend on the choice (each unit's
+ * arithmetic is the same either way).
  */
 FA_API size_t fa_fwd_workspace_size(int B, int Hq, int Hkv, int Sq, int Sk, int D);
 FA_API int fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -111,7 +117,7 @@ FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* out, 
  * = total_*.  Both arrays are DEVICE int32 [num_seqs + 1].  max_seqlen_* must
  * bound every sequence length (they size the grid).
  *   q, out [total_q, Hq, D]    k, v [total_k, Hkv, D]    lse [Hq, total_q] float32
- * Workspace: none.
+ * Workspace: optional, as for fa_fwd (the dynamic schedule balances unequal lengths).
  */
 FA_API size_t fa_varlen_fwd_workspace_size(int num_seqs, int total_q, int total_k, int Hq, int Hkv, int D);
 FA_API int fa_varlen_fwd(const void* q, const void* k, const void* v, void* out, float* lse,

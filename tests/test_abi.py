@@ -114,8 +114,19 @@ def test_varlen_rejects_missing_cu_seqlens(lib):
     assert st == abi.FA_ERR_INVALID_ARG
     st = abi.fa_varlen_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 2, 2, 10, 10, 20, 20, 2, 2, 64, 0.1, 1, stream=S0)
     assert st == abi.FA_ERR_ALIGNMENT
-    assert abi.fa_varlen_fwd_workspace_size(2, 20, 20, 2, 2, 64) == 0
+    assert abi.fa_varlen_fwd_workspace_size(2, 20, 20, 2, 2, 64) == 256
     assert abi.fa_varlen_bwd_workspace_size(2, 20, 20, 2, 2, 64) > 0
+
+
+def test_forward_workspace_is_optional_but_checked(lib):
+    # 256 bytes for the dynamic schedule's unit counter; NULL selects the static schedule, and a given
+    # workspace must follow the usual rules (size, 256-byte alignment) -- checked before any launch
+    assert abi.fa_fwd_workspace_size(2, 4, 2, 100, 100, 64) == 256
+    args = (FAKE, FAKE, FAKE, FAKE, FAKE, 2, 4, 2, 100, 100, 64, 0.1, 1)
+    assert abi.fa_fwd(*args, FAKE, 255, S0) == abi.FA_ERR_WORKSPACE
+    assert abi.fa_fwd(*args, FAKE + 16, 256, S0) == abi.FA_ERR_ALIGNMENT
+    vargs = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 2, 10, 10, 20, 20, 2, 2, 64, 0.1, 1)
+    assert abi.fa_varlen_fwd(*vargs, FAKE, 100, S0) == abi.FA_ERR_WORKSPACE
 
 
 def test_kvcache_argument_rules(lib):
