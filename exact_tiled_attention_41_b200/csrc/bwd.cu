@@ -310,6 +310,19 @@ __global__ void __launch_bounds__(512, 1)
                 constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
                 constexpr uint32_t id_tn = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
                 constexpr uint32_t id_dq = idesc_bf16_f32(128, D, true, true);       // dQ, all D columns
+                // Descriptor low words, advanced by constant offsets >> 4: one add per operand per MMA, so the
+                // issuing thread keeps up with the tensor core (about 54 cycles per MMA at best from one
+                // thread, against 64 for these 128 x 128 x 16 steps)
+                constexpr uint32_t T16 = C::T_BYTES >> 4, ROWS16 = (16 * 128) >> 4;
+                const uint32_t dK0 = sdesc_lo(smem_u32(smem + C::OFF_K), 16);             // K, K-major
+                const uint32_t dV0 = sdesc_lo(smem_u32(smem + C::OFF_V), 16);             // V, K-major
+                const uint32_t dQ0 = sdesc_lo(smem_u32(smem + C::OFF_Q), 16);             // Q stage 0, K-major
+                const uint32_t dO0 = sdesc_lo(smem_u32(smem + C::OFF_DO), 16);            // dO stage 0, K-major
+                const uint32_t dQ0n = sdesc_lo(smem_u32(smem + C::OFF_Q), 128 * 128);     // Q as MN-major B
+                const uint32_t dO0n = sdesc_lo(smem_u32(smem + C::OFF_DO), 128 * 128);    // dO as MN-major B
+                const uint32_t dSn = sdesc_lo(smem_u32(smem + C::OFF_DS), 128 * 128);     // dS, MN-major A of dQ
+                const uint32_t dKn = sdesc_lo(smem_u32(smem + C::OFF_K), 128 * 128);      // K, MN-major B of dQ
+                auto kchunk = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4); };
                 uint32_t unit_it = 0, q_it = 0, g_it = 0;
                 bool ok = true;
                 for (uint32_t fi = 0; ok; ++fi) {
@@ -325,59 +338,45 @@ __global__ void __launch_bounds__(512, 1)
                         const int st = q_it % ST;
                         if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
                         tc_fence_after();
-                        const uint8_t* sq = smem + C::OFF_Q + st * C::T_BYTES;
-                        const uint8_t* sdo = smem + C::OFF_DO + st * C::T_BYTES;
+                        const uint32_t qd = dQ0 + st * T16, od = dO0 + st * T16;
+                        const uint32_t qn = dQ0n + st * T16, on = dO0n + st * T16;
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                            umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + o), 16, 1024),
-                                    sdesc_sw128(smem_u32(sq + o), 16, 1024), id_kk, kk > 0);
-                        }
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lo(tmem + C::COL_S, dK0 + kchunk(kk), qd + kchunk(kk), id_kk, kk > 0);
                         if (!DQ && last) umma_commit(k_free);     // K's last reader without the dQ product
                         // dP^T goes where the previous tile's dQ was: both halves of it must be read out
                         if (DQ && g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
                         if (DQ && g_it > 0 && !mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t o = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                            umma_ss(tmem + C::COL_DP, sdesc_sw128(smem_u32(smem + C::OFF_V + o), 16, 1024),
-                                    sdesc_sw128(smem_u32(sdo + o), 16, 1024), id_kk, kk > 0);
-                        }
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lo(tmem + C::COL_DP, dV0 + kchunk(kk), od + kchunk(kk), id_kk, kk > 0);
                         umma_commit(s_full);
                         if (last) umma_commit(v_free);            // V's last reader in this unit
                         // dV += P^T dO, dK += dS^T Q over queries 0-63, as soon as warpgroup 0 is done
                         if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
+                        const uint32_t first = it > 0 ? 1u : 0u;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                            umma_ts(tmem + C::COL_DV, tmem + C::COL_P(kk),
-                                    sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
-                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DSP(kk),
-                                    sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, acc);
+                            umma_ts_lo(tmem + C::COL_DV, tmem + C::COL_P(kk), on + kk * ROWS16, id_tn, kk > 0 ? 1u : first);
+                            umma_ts_lo(tmem + C::COL_DK, tmem + C::COL_DSP(kk), qn + kk * ROWS16, id_tn, kk > 0 ? 1u : first);
                         }
                         if (!mbar_wait(p_full_hi, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
                         if constexpr (DQ) {
                             // dQ = dS K over dP^T's columns (read out by the dQ warpgroup while dV / dK finish)
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) {     // K-dim = 128 key rows
-                                umma_ss(tmem + C::COL_DQ,
-                                        sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
-                                        sdesc_sw128(smem_u32(smem + C::OFF_K + kk * 16 * 128), 128 * 128, 1024),
-                                        id_dq, kk > 0);
-                            }
+                            for (int kk = 0; kk < 8; ++kk)     // K-dim = 128 key rows
+                                umma_ss_lo(tmem + C::COL_DQ, dSn + kk * ROWS16, dKn + kk * ROWS16, id_dq, kk > 0);
                             umma_commit(dq_full);
                             if (last) umma_commit(k_free);        // K's last reader in this unit
                         }
                         // dV, dK over queries 64-127
 #pragma unroll
                         for (int kk = 4; kk < 8; ++kk) {
-                            umma_ts(tmem + C::COL_DV, tmem + C::COL_P(kk),
-                                    sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 128 * 128, 1024), id_tn, 1u);
-                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DSP(kk),
-                                    sdesc_sw128(smem_u32(sq + kk * 16 * 128), 128 * 128, 1024), id_tn, 1u);
+                            umma_ts_lo(tmem + C::COL_DV, tmem + C::COL_P(kk), on + kk * ROWS16, id_tn, 1u);
+                            umma_ts_lo(tmem + C::COL_DK, tmem + C::COL_DSP(kk), qn + kk * ROWS16, id_tn, 1u);
                         }
                         umma_commit(q_empty(st));
                     }
@@ -796,6 +795,14 @@ __global__ void __launch_bounds__(384, 1)
             if (lane == 0) {
                 constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);    // S^T, dP^T of an item
                 constexpr uint32_t id_t = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
+                // descriptor low words advanced by constant offsets >> 4 (one add per operand per MMA)
+                constexpr uint32_t IT16 = C::IT_BYTES >> 4, ROWS16 = (16 * 128) >> 4;
+                const uint32_t dK0 = sdesc_lo(smem_u32(smem + C::OFF_K), 16), dV0 = sdesc_lo(smem_u32(smem + C::OFF_V), 16);
+                const uint32_t dQ0 = sdesc_lo(smem_u32(smem + C::OFF_Q), 16), dO0 = sdesc_lo(smem_u32(smem + C::OFF_DO), 16);
+                const uint32_t dQ0n = sdesc_lo(smem_u32(smem + C::OFF_Q), 64 * 128);
+                const uint32_t dO0n = sdesc_lo(smem_u32(smem + C::OFF_DO), 64 * 128);
+                auto achunk = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4); };
+                auto bchunk = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * 64 * 128 + (kk & 3) * 32) >> 4); };
                 uint32_t unit_it = 0, q_it = 0, gi = 0;
                 bool ok = true;
                 // dV, dK of item g (buffer g % 2, stage st); `first`: the unit's first item overwrites dV, dK
@@ -805,15 +812,12 @@ __global__ void __launch_bounds__(384, 1)
                     // the previous unit's epilogues must have read dV and dK before they are overwritten
                     if (first && unit_it > 0 && !mbar_wait(dkv_empty, (unit_it - 1) & 1, w)) return false;
                     tc_fence_after();
-                    const uint8_t* sq = smem + C::OFF_Q + st * C::IT_BYTES;
-                    const uint8_t* sdo = smem + C::OFF_DO + st * C::IT_BYTES;
+                    const uint32_t qn = dQ0n + st * IT16, on = dO0n + st * IT16;
+                    const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {     // K-dim = 64 item queries
-                        const uint32_t acc = (!first || kk > 0) ? 1u : 0u;
-                        umma_ts(tmem + C::COL_DV, tmem + C::COL_P(b, kk),
-                                sdesc_sw128(smem_u32(sdo + kk * 16 * 128), 64 * 128, 1024), id_t, acc);
-                        umma_ts(tmem + C::COL_DK, tmem + C::COL_DSP(b, kk),
-                                sdesc_sw128(smem_u32(sq + kk * 16 * 128), 64 * 128, 1024), id_t, acc);
+                        umma_ts_lo(tmem + C::COL_DV, tmem + C::COL_P(b, kk), on + kk * ROWS16, id_t, kk > 0 ? 1u : acc0);
+                        umma_ts_lo(tmem + C::COL_DK, tmem + C::COL_DSP(b, kk), qn + kk * ROWS16, id_t, kk > 0 ? 1u : acc0);
                     }
                     umma_commit(q_empty(st));
                     return true;
@@ -831,22 +835,13 @@ __global__ void __launch_bounds__(384, 1)
                         const int b = gi & 1;
                         if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
                         tc_fence_after();
-                        const uint8_t* sq = smem + C::OFF_Q + st * C::IT_BYTES;
-                        const uint8_t* sdo = smem + C::OFF_DO + st * C::IT_BYTES;
+                        const uint32_t qd = dQ0 + st * IT16, od = dO0 + st * IT16;
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oa = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                            const uint32_t ob = (kk >> 2) * 64 * 128 + (kk & 3) * 32;
-                            umma_ss(tmem + C::COL_S(b), sdesc_sw128(smem_u32(smem + C::OFF_K + oa), 16, 1024),
-                                    sdesc_sw128(smem_u32(sq + ob), 16, 1024), id_s, kk > 0);
-                        }
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lo(tmem + C::COL_S(b), dK0 + achunk(kk), qd + bchunk(kk), id_s, kk > 0);
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t oa = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                            const uint32_t ob = (kk >> 2) * 64 * 128 + (kk & 3) * 32;
-                            umma_ss(tmem + C::COL_DP(b), sdesc_sw128(smem_u32(smem + C::OFF_V + oa), 16, 1024),
-                                    sdesc_sw128(smem_u32(sdo + ob), 16, 1024), id_s, kk > 0);
-                        }
+                        for (int kk = 0; kk < D / 16; ++kk)
+                            umma_ss_lo(tmem + C::COL_DP(b), dV0 + achunk(kk), od + bchunk(kk), id_s, kk > 0);
                         umma_commit(s_full(b));
                         // the previous item's products, while warpgroup b works on this one
                         if (i > 0 && !post(prev_g, prev_st, i == 1)) { ok = false; break; }

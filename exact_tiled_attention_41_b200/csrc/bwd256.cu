@@ -7,7 +7,8 @@
 // head dimension of dV and dK.  The unit still contracts S^T = K Q^T and
 // dP^T = V dO^T over the full head dimension (the two halves recompute them),
 // and emits the matching half of dQ.  Query tiles are 64 rows so that K, V
-// (128 x 256 each), Q, dO (64 x 256) and dS^T fit shared memory.
+// (128 x 256 each), a ring of five 16 KB slots for the Q and dO tiles (see Cfg)
+// and dS^T fit shared memory.
 //   tensor memory: dV half [0,128) | dK half [128,256) | S^T [256,320) |
 //                  dP^T [320,384) | dQ^T half [384,448)
 //   dQ^T = K_half^T dS^T has the head dimension on the 128 lanes, so the dQ
@@ -21,6 +22,10 @@
 #include "sm100.cuh"
 
 #include <math.h>
+
+#ifndef FA_B256_VEC_DQ
+#define FA_B256_VEC_DQ 1
+#endif
 
 namespace fa {
 
@@ -97,14 +102,26 @@ __device__ __forceinline__ U256 decode_u256(const B256Params& p, int u) {
     return t;
 }
 
+// Q and dO of a 64-row query tile arrive as four pairs of [64 x 64] boxes (two head-dim chunks each),
+// in this order: Q of the other half, dO of the other half, Q of the unit's half, dO of the unit's half.
+// The pairs pass through a ring of NSLOT 16 KB slots and each slot is released by the last product that
+// reads it (S^T; dP^T; dK; dV), so the next tile's S^T operands and half of its dP^T operands load
+// while the current tile's gradient step runs.
 struct Cfg {
     static constexpr uint32_t KV_BYTES = 128 * D * 2;    // 64 KB, four [128 x 64] boxes
-    static constexpr uint32_t QT_BYTES = 64 * D * 2;     // 32 KB, four [64 x 64] boxes
-    static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_Q = 2 * KV_BYTES, OFF_DO = OFF_Q + QT_BYTES,
-                              OFF_DS = OFF_DO + QT_BYTES,               // dS^T [128 keys][64 queries], 16 KB
-                              OFF_STAT = OFF_DS + 128 * 128, OFF_BAR = OFF_STAT + 2 * 64 * 4;
-    static constexpr int NUM_BARS = 9 + 2 * kFeedSlots;
+    static constexpr uint32_t BOX_BYTES = 64 * 64 * 2, PAIR_BYTES = 2 * BOX_BYTES;
+    static constexpr uint32_t NSLOT = 5;
+    static constexpr uint32_t OFF_K = 0, OFF_V = KV_BYTES, OFF_RING = 2 * KV_BYTES,
+                              OFF_DS = OFF_RING + NSLOT * PAIR_BYTES,   // dS^T [128 keys][64 queries], 16 KB
+                              OFF_STAT = OFF_DS + 128 * 128,            // [2][-LSE2 x 64 | -Delta x 64]
+                              OFF_BAR = OFF_STAT + 2 * 128 * 4;
+    // kv_full, kv_empty | slot_full[NSLOT] | slot_empty[NSLOT] | stat_full[2] | stat_empty[2] |
+    // s_full, p_full, dq_full, dq_empty, dkv_full | unit feed
+    static constexpr int BAR_SLOT_FULL = 2, BAR_SLOT_EMPTY = 2 + NSLOT, BAR_STAT_FULL = 2 + 2 * NSLOT,
+                         BAR_STAT_EMPTY = BAR_STAT_FULL + 2, BAR_S_FULL = BAR_STAT_EMPTY + 2, BAR_FEED = BAR_S_FULL + 5;
+    static constexpr int NUM_BARS = BAR_FEED + 2 * kFeedSlots;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
+    static_assert(SMEM <= 232448, "shared memory per block");
     static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
     static constexpr int THREADS = 384, LAUNCH_REGS = 168, COMPUTE_REGS = 232, OTHER_REGS = 136;
     static_assert(128 * COMPUTE_REGS + 2 * 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
@@ -117,16 +134,20 @@ __global__ void __launch_bounds__(384, 1)
                   const __grid_constant__ B256Params p) {
     using C = Cfg;
     extern __shared__ __align__(1024) uint8_t smem[];
-    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_STAT);   // [64]
-    float* sDel = sLSE + 64;                                      // [64]
+    float* sStat = reinterpret_cast<float*>(smem + C::OFF_STAT);  // [2][128]: -LSE2 of 64 rows, -Delta of 64 rows
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* feed_slot = reinterpret_cast<int*>(tmem_slot + 4);
     const uint32_t b0 = smem_u32(bars);
-    const UnitFeed feed{feed_slot, b0 + 8u * 9, b0 + 8u * (9 + kFeedSlots)};
-    const uint32_t kv_full = b0, kv_empty = b0 + 8, q_full = b0 + 16, q_empty = b0 + 24, s_full = b0 + 32,
-                   p_full = b0 + 40, dq_full = b0 + 48, dq_empty = b0 + 56, dkv_full = b0 + 64;
+    const UnitFeed feed{feed_slot, b0 + 8u * C::BAR_FEED, b0 + 8u * (C::BAR_FEED + kFeedSlots)};
+    const uint32_t kv_full = b0, kv_empty = b0 + 8;
+    auto slot_full = [&](uint32_t s) { return b0 + 8u * (C::BAR_SLOT_FULL + s); };
+    auto slot_empty = [&](uint32_t s) { return b0 + 8u * (C::BAR_SLOT_EMPTY + s); };
+    auto stat_full = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_FULL + s); };
+    auto stat_empty = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_EMPTY + s); };
+    const uint32_t s_full = b0 + 8u * C::BAR_S_FULL, p_full = s_full + 8, dq_full = s_full + 16,
+                   dq_empty = s_full + 24, dkv_full = s_full + 32;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PRODUCER = 8, MMA = 9;
 
@@ -135,18 +156,24 @@ __global__ void __launch_bounds__(384, 1)
         return;
     }
     if (threadIdx.x == 0) {
-        mbar_init(bars + 0, 1);
-        mbar_init(bars + 1, 1);
-        mbar_init(bars + 2, 33);     // q_full: 32 producer lanes (statistics) + the TMA expect-tx arrival
-        mbar_init(bars + 3, 1);
-        mbar_init(bars + 4, 1);
-        mbar_init(bars + 5, 128);    // p_full
-        mbar_init(bars + 6, 1);
-        mbar_init(bars + 7, 128);    // dq_empty
-        mbar_init(bars + 8, 1);
+        mbar_init(bars + 0, 1);                                      // kv_full
+        mbar_init(bars + 1, 1);                                      // kv_empty
+        for (int s = 0; s < static_cast<int>(C::NSLOT); ++s) {
+            mbar_init(bars + C::BAR_SLOT_FULL + s, 1);               // expect-tx arrival of the pair's loads
+            mbar_init(bars + C::BAR_SLOT_EMPTY + s, 1);              // commit of the pair's last reader
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bars + C::BAR_STAT_FULL + s, 32);              // the producer's 32 lanes
+            mbar_init(bars + C::BAR_STAT_EMPTY + s, 4);              // one arrival per compute warp
+        }
+        mbar_init(bars + C::BAR_S_FULL + 0, 1);                      // s_full
+        mbar_init(bars + C::BAR_S_FULL + 1, 128);                    // p_full
+        mbar_init(bars + C::BAR_S_FULL + 2, 1);                      // dq_full
+        mbar_init(bars + C::BAR_S_FULL + 3, 128);                    // dq_empty
+        mbar_init(bars + C::BAR_S_FULL + 4, 1);                      // dkv_full
         for (int s = 0; s < kFeedSlots; ++s) {
-            mbar_init(bars + 9 + s, 1);                              // unit published
-            mbar_init(bars + 9 + kFeedSlots + s, DQ ? 9 : 5);        // read by MMA, compute (, dQ) warps
+            mbar_init(bars + C::BAR_FEED + s, 1);                              // unit published
+            mbar_init(bars + C::BAR_FEED + kFeedSlots + s, DQ ? 9 : 5);        // read by MMA, compute (, dQ) warps
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -173,6 +200,18 @@ __global__ void __launch_bounds__(384, 1)
         if (warp == PRODUCER) {
             uint32_t unit_it = 0, q_it = 0;
             bool ok = true;
+            // head-dim chunks c0, c0 + 1 of a 64-row tile of Q or dO into the ring slot of pair number px
+            auto load_pair = [&](uint32_t px, const CUtensorMap* map, int c0, int h, int row) -> bool {
+                const uint32_t sl = px % C::NSLOT, n = px / C::NSLOT;
+                if (n > 0 && !mbar_wait(slot_empty(sl), (n - 1) & 1, w)) return false;
+                if (lane == 0) {
+                    const uint32_t dst = smem_u32(smem + C::OFF_RING + sl * C::PAIR_BYTES);
+                    mbar_arrive_expect_tx(slot_full(sl), C::PAIR_BYTES);
+                    tma_load_3d(dst, map, slot_full(sl), c0 * 64, h, row);
+                    tma_load_3d(dst + C::BOX_BYTES, map, slot_full(sl), (c0 + 1) * 64, h, row);
+                }
+                return true;
+            };
             for (uint32_t fi = 0; ok; ++fi) {
                 int u = 0;
                 if (lane == 0 && !feed_put(feed, fi, p.counter, p.num_units, u, w)) u = -2;
@@ -181,43 +220,53 @@ __global__ void __launch_bounds__(384, 1)
                 if (u < 0) break;
                 const U256 t = decode_u256(p, u);
                 if (t.skip || t.n_it == 0) continue;
-                if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(kv_full, 2 * C::KV_BYTES);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
-                                    t.k_start + t.n0);
-                        tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
-                                    t.k_start + t.n0);
-                    }
-                }
-                ++unit_it;
+                const int oh = 1 - t.hh;
                 for (int it = 0; it < t.n_it; ++it, ++q_it) {
                     const int g = it / t.n_m;
                     const int m0 = (t.m_start + it % t.n_m) * 64;
                     const int h = t.hk * G + g;
-                    if (q_it > 0 && !mbar_wait(q_empty, (q_it - 1) & 1, w)) { ok = false; break; }
+                    const int row = t.q_start + m0;
+                    // the tile's statistics into registers first, so their loads overlap the waits below;
+                    // rows past the sequence get -LSE2 = -inf (P = 0) and Delta = 0; stored negated
+                    float nl[2], nd[2];
 #pragma unroll
                     for (int e = 0; e < 2; ++e) {
-                        const int qi = lane * 2 + e;
-                        const int row = m0 + qi;
-                        const bool in = row < t.Lq;
-                        const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + row;
-                        sLSE[qi] = in ? __ldg(p.lse2 + idx) : INFINITY;
-                        sDel[qi] = in ? __ldg(p.delta + idx) : 0.f;
+                        const int rr = m0 + lane * 2 + e;
+                        const bool in = rr < t.Lq;
+                        const size_t idx = static_cast<size_t>(h) * p.Tq + t.q_start + rr;
+                        nl[e] = in ? -__ldg(p.lse2 + idx) : -INFINITY;
+                        nd[e] = in ? -__ldg(p.delta + idx) : 0.f;
                     }
-                    if (lane == 0) {
-                        mbar_arrive_expect_tx(q_full, 2 * C::QT_BYTES);
+                    const uint32_t px = 4u * q_it;
+                    if (!load_pair(px, &tmQ, 2 * oh, h, row) || !load_pair(px + 1, &tmDO, 2 * oh, h, row) ||
+                        !load_pair(px + 2, &tmQ, 2 * t.hh, h, row)) {
+                        ok = false;
+                        break;
+                    }
+                    if (it == 0) {
+                        // K and V of the unit, once the previous unit's last products have run
+                        if (unit_it > 0 && !mbar_wait(kv_empty, (unit_it - 1) & 1, w)) { ok = false; break; }
+                        if (lane == 0) {
+                            mbar_arrive_expect_tx(kv_full, 2 * C::KV_BYTES);
 #pragma unroll
-                        for (int c = 0; c < 4; ++c) {
-                            tma_load_3d(smem_u32(smem + C::OFF_Q + c * 64 * 128), &tmQ, q_full, c * 64, h,
-                                        t.q_start + m0);
-                            tma_load_3d(smem_u32(smem + C::OFF_DO + c * 64 * 128), &tmDO, q_full, c * 64, h,
-                                        t.q_start + m0);
+                            for (int c = 0; c < 4; ++c) {
+                                tma_load_3d(smem_u32(smem + C::OFF_K + c * 128 * 128), &tmK, kv_full, c * 64, t.hk,
+                                            t.k_start + t.n0);
+                                tma_load_3d(smem_u32(smem + C::OFF_V + c * 128 * 128), &tmV, kv_full, c * 64, t.hk,
+                                            t.k_start + t.n0);
+                            }
                         }
+                        ++unit_it;
                     }
-                    mbar_arrive(q_full);
+                    if (!load_pair(px + 3, &tmDO, 2 * t.hh, h, row)) { ok = false; break; }
+                    const uint32_t sb = q_it & 1;
+                    if (q_it >= 2 && !mbar_wait(stat_empty(sb), ((q_it >> 1) - 1) & 1, w)) { ok = false; break; }
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        sStat[sb * 128 + lane * 2 + e] = nl[e];
+                        sStat[sb * 128 + 64 + lane * 2 + e] = nd[e];
+                    }
+                    mbar_arrive(stat_full(sb));
                 }
             }
             __syncwarp();
@@ -226,6 +275,16 @@ __global__ void __launch_bounds__(384, 1)
                 constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);     // S^T, dP^T
                 constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, true);     // dV, dK halves
                 constexpr uint32_t id_q = idesc_bf16_f32(128, 64, true, true);       // dQ^T half
+                // Descriptor low words, advanced by constant offsets >> 4 (one add per operand per MMA: the
+                // issuing thread needs about as long per MMA as the tensor core at N = 64, so the loop is kept
+                // free of any other arithmetic)
+                constexpr uint32_t CHUNK16 = (128 * 128) >> 4, BOX16 = C::BOX_BYTES >> 4, PAIR16 = C::PAIR_BYTES >> 4,
+                                   K16 = 32 >> 4, ROWS16 = (16 * 128) >> 4;
+                const uint32_t dK0 = sdesc_lo(smem_u32(smem + C::OFF_K), 16);           // K, K-major boxes
+                const uint32_t dV0 = sdesc_lo(smem_u32(smem + C::OFF_V), 16);           // V
+                const uint32_t dDS = sdesc_lo(smem_u32(smem + C::OFF_DS), 128 * 128);   // dS^T, dQ^T's B (MN-major)
+                const uint32_t dRK = sdesc_lo(smem_u32(smem + C::OFF_RING), 16);        // ring pairs, K-major
+                const uint32_t dRN = sdesc_lo(smem_u32(smem + C::OFF_RING), C::BOX_BYTES);   // ring pairs, MN-major
                 uint32_t unit_it = 0, q_it = 0;
                 bool ok = true;
                 for (uint32_t fi = 0; ok; ++fi) {
@@ -235,23 +294,57 @@ __global__ void __launch_bounds__(384, 1)
                     const U256 t = decode_u256(p, u);
                     if (t.skip || t.n_it == 0) continue;
                     if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
+                    const int oh = 1 - t.hh;
+                    const uint32_t kO = dK0 + 2 * oh * CHUNK16, kH = dK0 + 2 * t.hh * CHUNK16;
+                    const uint32_t vO = dV0 + 2 * oh * CHUNK16, vH = dV0 + 2 * t.hh * CHUNK16;
+                    // K[:, half]^T as dQ^T's A operand (MN-major: the two 64-column boxes of the half, 16 KB apart)
+                    const uint32_t kT = sdesc_lo(smem_u32(smem + C::OFF_K + 2 * t.hh * 128 * 128), 128 * 128);
                     for (int it = 0; it < t.n_it; ++it, ++q_it) {
-                        if (!mbar_wait(q_full, q_it & 1, w)) { ok = false; break; }
+                        // ring slots of the tile's pairs: Q other half, dO other half, Q own half, dO own half
+                        const uint32_t px = 4u * q_it;
+                        uint32_t sl[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) sl[k] = (px + k) % C::NSLOT;
+                        auto pair_ready = [&](int k) {
+                            return mbar_wait(slot_full(sl[k]), ((px + k) / C::NSLOT) & 1, w);
+                        };
+                        const uint32_t q0 = dRK + sl[0] * PAIR16, o1 = dRK + sl[1] * PAIR16,
+                                       q2 = dRK + sl[2] * PAIR16, o3 = dRK + sl[3] * PAIR16;
+                        const uint32_t q2n = dRN + sl[2] * PAIR16, o3n = dRN + sl[3] * PAIR16;
+                        if (!pair_ready(0) || !pair_ready(2)) { ok = false; break; }
+                        tc_fence_after();
+                        // S^T = K Q^T over the head dim, the other half's chunks first
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; ++k4)
+                                umma_ss_lo(tmem + C::COL_S, kO + i * CHUNK16 + k4 * K16, q0 + i * BOX16 + k4 * K16, id_s,
+                                           (i | k4) != 0);
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; ++k4)
+                                umma_ss_lo(tmem + C::COL_S, kH + i * CHUNK16 + k4 * K16, q2 + i * BOX16 + k4 * K16, id_s,
+                                           1u);
+                        umma_commit(slot_empty(sl[0]));           // Q of the other half: last read by S^T
+                        if (!pair_ready(1)) { ok = false; break; }
+                        tc_fence_after();
+                        // dP^T = V dO^T, the other half first (its pair is loaded early), then the own half
+#pragma unroll
+                        for (int i = 0; i < 2; ++i)
+#pragma unroll
+                            for (int k4 = 0; k4 < 4; ++k4)
+                                umma_ss_lo(tmem + C::COL_DP, vO + i * CHUNK16 + k4 * K16, o1 + i * BOX16 + k4 * K16, id_s,
+                                           (i | k4) != 0);
+                        umma_commit(slot_empty(sl[1]));           // dO of the other half: last read by dP^T
+                        if (!pair_ready(3)) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t ok_ = (kk >> 2) * 128 * 128 + (kk & 3) * 32;   // [128 x 64] boxes
-                            const uint32_t oq = (kk >> 2) * 64 * 128 + (kk & 3) * 32;      // [64 x 64] boxes
-                            umma_ss(tmem + C::COL_S, sdesc_sw128(smem_u32(smem + C::OFF_K + ok_), 16, 1024),
-                                    sdesc_sw128(smem_u32(smem + C::OFF_Q + oq), 16, 1024), id_s, kk > 0);
-                        }
+                        for (int i = 0; i < 2; ++i)
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t ok_ = (kk >> 2) * 128 * 128 + (kk & 3) * 32;
-                            const uint32_t oq = (kk >> 2) * 64 * 128 + (kk & 3) * 32;
-                            umma_ss(tmem + C::COL_DP, sdesc_sw128(smem_u32(smem + C::OFF_V + ok_), 16, 1024),
-                                    sdesc_sw128(smem_u32(smem + C::OFF_DO + oq), 16, 1024), id_s, kk > 0);
-                        }
+                            for (int k4 = 0; k4 < 4; ++k4)
+                                umma_ss_lo(tmem + C::COL_DP, vH + i * CHUNK16 + k4 * K16, o3 + i * BOX16 + k4 * K16, id_s,
+                                           1u);
                         umma_commit(s_full);
                         if (!mbar_wait(p_full, q_it & 1, w)) { ok = false; break; }
                         if (DQ && q_it > 0 && !mbar_wait(dq_empty, (q_it - 1) & 1, w)) { ok = false; break; }
@@ -259,29 +352,23 @@ __global__ void __launch_bounds__(384, 1)
                         if constexpr (DQ) {
                             // dQ^T half = K[:, half]^T dS^T (K-dim = 128 keys)
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) {
-                                umma_ss(tmem + C::COL_DQ,
-                                        sdesc_sw128(smem_u32(smem + C::OFF_K + 2 * t.hh * 128 * 128 + kk * 16 * 128),
-                                                    128 * 128, 1024),
-                                        sdesc_sw128(smem_u32(smem + C::OFF_DS + kk * 16 * 128), 128 * 128, 1024),
-                                        id_q, kk > 0);
-                            }
+                            for (int kk = 0; kk < 8; ++kk)
+                                umma_ss_lo(tmem + C::COL_DQ, kT + kk * ROWS16, dDS + kk * ROWS16, id_q, kk > 0);
                             umma_commit(dq_full);
                         }
-                        // dV half += P^T dO[:, half], dK half += dS^T Q[:, half] (K-dim = 64 queries)
+                        // dK half += dS^T Q[:, half], then dV half += P^T dO[:, half] (K-dim = 64 queries): the
+                        // own-half Q pair is released first, because the next tile's last pair waits for its slot
+                        const uint32_t first = it > 0 ? 1u : 0u;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint32_t acc = (it > 0 || kk > 0) ? 1u : 0u;
-                            umma_ts(tmem + C::COL_DV, tmem + C::COL_S + kk * 8,
-                                    sdesc_sw128(smem_u32(smem + C::OFF_DO + 2 * t.hh * 64 * 128 + kk * 16 * 128),
-                                                64 * 128, 1024),
-                                    id_g, acc);
-                            umma_ts(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8,
-                                    sdesc_sw128(smem_u32(smem + C::OFF_Q + 2 * t.hh * 64 * 128 + kk * 16 * 128),
-                                                64 * 128, 1024),
-                                    id_g, acc);
-                        }
-                        umma_commit(q_empty);
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_ts_lo(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, q2n + kk * ROWS16, id_g,
+                                       kk > 0 ? 1u : first);
+                        umma_commit(slot_empty(sl[2]));
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_ts_lo(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, o3n + kk * ROWS16, id_g,
+                                       kk > 0 ? 1u : first);
+                        umma_commit(slot_empty(sl[3]));
                     }
                     if (!ok) break;
                     umma_commit(dkv_full);
@@ -293,7 +380,6 @@ __global__ void __launch_bounds__(384, 1)
         } else if (DQ && warp < 8) {
             // -------------------------------------------------------- dQ warpgroup (thread = head-dim row)
             const int wq = warp - 4;
-            const int r = wq * 32 + lane;
             const uint32_t lb = tmem_lane_base(wq);
             uint32_t q_it = 0;
             bool ok = true;
@@ -309,7 +395,43 @@ __global__ void __launch_bounds__(384, 1)
                     const int h = t.hk * G + g;
                     if (!mbar_wait(dq_full, q_it & 1, w)) { ok = false; break; }
                     tc_fence_after();
-                    float* acc = p.dq_acc + (static_cast<size_t>(h) * p.Tq + t.q_start + m0) * D + t.hh * 128 + r;
+#if FA_B256_VEC_DQ
+                    // lanes 4g .. 4g+3 hold head-dim rows 4g .. 4g+3; a 4 x 4 transpose across them (two
+                    // butterfly steps) gives lane 4g+j the four head-dim values of query 4b+j, which leave
+                    // as one 16-byte reduce-add (8 rows of 128 bytes per warp instruction)
+                    const int j4 = lane & 3;
+                    float* acc = p.dq_acc + (static_cast<size_t>(h) * p.Tq + t.q_start + m0) * D + t.hh * 128 +
+                                 wq * 32 + (lane & ~3);
+#pragma unroll 1
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint32_t ra[32];
+                        tmem_ld32(tmem + lb + C::COL_DQ + cc * 32, ra);
+                        tmem_ld_wait_tie(ra);
+#pragma unroll
+                        for (int b4 = 0; b4 < 8; ++b4) {
+                            float v0 = __uint_as_float(ra[4 * b4]), v1 = __uint_as_float(ra[4 * b4 + 1]),
+                                  v2 = __uint_as_float(ra[4 * b4 + 2]), v3 = __uint_as_float(ra[4 * b4 + 3]);
+                            {
+                                const bool hi = (j4 & 1) != 0;
+                                const float y0 = __shfl_xor_sync(0xffffffffu, hi ? v0 : v1, 1);
+                                const float y1 = __shfl_xor_sync(0xffffffffu, hi ? v2 : v3, 1);
+                                if (hi) { v0 = y0; v2 = y1; } else { v1 = y0; v3 = y1; }
+                            }
+                            {
+                                const bool hi = (j4 & 2) != 0;
+                                const float y0 = __shfl_xor_sync(0xffffffffu, hi ? v0 : v2, 2);
+                                const float y1 = __shfl_xor_sync(0xffffffffu, hi ? v1 : v3, 2);
+                                if (hi) { v0 = y0; v1 = y1; } else { v2 = y0; v3 = y1; }
+                            }
+                            const int qc = cc * 32 + 4 * b4 + j4;
+                            if (m0 + qc < t.Lq)
+                                atomicAdd(reinterpret_cast<float4*>(acc + static_cast<size_t>(qc) * D),
+                                          make_float4(v0, v1, v2, v3));
+                        }
+                    }
+#else
+                    float* acc =
+                        p.dq_acc + (static_cast<size_t>(h) * p.Tq + t.q_start + m0) * D + t.hh * 128 + wq * 32 + lane;
 #pragma unroll 1
                     for (int cc = 0; cc < 2; ++cc) {
                         uint32_t ra[32];
@@ -321,6 +443,7 @@ __global__ void __launch_bounds__(384, 1)
                             if (m0 + qc < t.Lq) atomicAdd(acc + static_cast<size_t>(qc) * D, __uint_as_float(ra[e]));
                         }
                     }
+#endif
                     tc_fence_before();
                     mbar_arrive(dq_empty);
                 }
@@ -360,7 +483,10 @@ __global__ void __launch_bounds__(384, 1)
             for (int it = 0; it < t.n_it; ++it, ++q_it) {
                 const int m0 = (t.m_start + it % t.n_m) * 64;
                 if (!mbar_wait(s_full, q_it & 1, w)) { ok = false; break; }
-                if (!mbar_wait(q_full, q_it & 1, w)) { ok = false; break; }
+                const uint32_t sb = q_it & 1;
+                if (!mbar_wait(stat_full(sb), (q_it >> 1) & 1, w)) { ok = false; break; }
+                const float* nL = sStat + sb * 128;      // -LSE2 of the tile's 64 rows
+                const float* nD = nL + 64;               // -Delta
                 tc_fence_after();
                 uint32_t sa[2][32], da[2][32];
                 tmem_ld32(tmem + lb + C::COL_S, sa[0]);
@@ -383,13 +509,13 @@ __global__ void __launch_bounds__(384, 1)
                         const int qc = half * 32 + e;
                         const float2 sv = make_float2(__uint_as_float(sa[half][e]), __uint_as_float(sa[half][e + 1]));
                         const float2 dv = make_float2(__uint_as_float(da[half][e]), __uint_as_float(da[half][e + 1]));
-                        const float2 a = ffma2(sv, c2v, make_float2(-sLSE[qc], -sLSE[qc + 1]));
+                        const float2 a = ffma2(sv, c2v, make_float2(nL[qc], nL[qc + 1]));
                         float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
                         if (any_mask) {
                             pr.x = (kvalid && qc >= qmin && qc <= qmax) ? pr.x : 0.f;
                             pr.y = (kvalid && qc + 1 >= qmin && qc + 1 <= qmax) ? pr.y : 0.f;
                         }
-                        const float2 ds = fmul2(pr, fadd2(dv, make_float2(-sDel[qc], -sDel[qc + 1])));
+                        const float2 ds = fmul2(pr, fadd2(dv, make_float2(nD[qc], nD[qc + 1])));
                         pp[e / 2] = pack_bf16x2(pr.x, pr.y);
                         dd[e / 2] = pack_bf16x2(ds.x, ds.y);
                     }
@@ -402,6 +528,8 @@ __global__ void __launch_bounds__(384, 1)
                             make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(stat_empty(sb));   // the warp has read the tile's statistics
                 tmem_st_wait();
                 fence_proxy_async_smem();
                 tc_fence_before();

@@ -222,25 +222,25 @@ __global__ void __launch_bounds__(384, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(BM, BK, false, false);   // S, dP: both K-major
             constexpr uint32_t idesc_dq = idesc_bf16_f32(BM, D, false, true);    // dQ: K tile N-major
-            // [128 x D] tile times a [BK x D] tile transposed, into tensor-memory column dcol
+            // [128 x D] tile times a [BK x D] tile transposed, into tensor-memory column dcol; descriptor
+            // low words advanced by constant offsets >> 4 (one add per operand per MMA)
             auto issue_ss = [&](uint32_t dcol, const uint8_t* a, const uint8_t* b) {
+                const uint32_t ad = sdesc_lo(smem_u32(a), 16), bd = sdesc_lo(smem_u32(b), 16);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ao = smem_u32(a + (kk >> 2) * BM * 128 + (kk & 3) * 32);
-                    const uint32_t bo = smem_u32(b + (kk >> 2) * BK * 128 + (kk & 3) * 32);
-                    umma_ss(tmem + dcol, sdesc_sw128(ao, 16, 1024), sdesc_sw128(bo, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma_ss_lo(tmem + dcol, ad + (((kk >> 2) * BM * 128 + (kk & 3) * 32) >> 4),
+                               bd + (((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4), idesc_s, kk > 0 ? 1u : 0u);
             };
             // dQ (+)= dS K: dS for keys [16 kk, 16 kk + 16) sits in the S half of the warpgroup that owns
             // those keys, at (key offset inside the half) / 2 packed columns from the half's start
             auto issue_dq = [&](int sb, int st, bool acc) {
+                const uint32_t kd = sdesc_lo(smem_u32(sK + st * C::KV_BYTES), BK * 128);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
                     const int k0 = kk * 16;
                     const uint32_t acol = C::S_COL(sb) + (k0 / HALF) * HALF + (k0 % HALF) / 2;
-                    const uint32_t kb = smem_u32(sK + st * C::KV_BYTES + kk * 16 * 128);
-                    umma_ts(tmem + C::DQ_COL, tmem + acol, sdesc_sw128(kb, BK * 128, 1024), idesc_dq,
-                            (acc || kk > 0) ? 1u : 0u);
+                    umma_ts_lo(tmem + C::DQ_COL, tmem + acol, kd + ((kk * 16 * 128) >> 4), idesc_dq,
+                               (acc || kk > 0) ? 1u : 0u);
                 }
             };
             uint32_t kv_it = 0, q_it = 0, gt = 0, unit_it = 0;

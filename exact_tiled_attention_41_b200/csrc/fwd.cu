@@ -355,19 +355,19 @@ __global__ void __launch_bounds__(FwdCfg<D, NQ, BK, KST>::THREADS, 1)
             // start-address field (shared-memory addresses stay below 2^18, so the 14-bit field never
             // carries): two adds per MMA, so the issuer keeps up with the tensor pipe
             auto issue_qk = [&](int i, int st) {
-                const uint64_t qd = sdesc_sw128(smem_u32(sQ + i * C::Q_BYTES), 16, 1024);
-                const uint64_t kd = sdesc_sw128(smem_u32(sK + st * C::KV_BYTES), 16, 1024);
+                const uint32_t qd = sdesc_lo(smem_u32(sQ + i * C::Q_BYTES), 16);
+                const uint32_t kd = sdesc_lo(smem_u32(sK + st * C::KV_BYTES), 16);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma_ss(tmem + C::S_COL(i), qd + (((kk >> 2) * BM * 128 + (kk & 3) * 32) >> 4),
-                            kd + (((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
+                    umma_ss_lo(tmem + C::S_COL(i), qd + (((kk >> 2) * BM * 128 + (kk & 3) * 32) >> 4),
+                               kd + (((kk >> 2) * BK * 128 + (kk & 3) * 32) >> 4), idesc_qk, kk > 0 ? 1u : 0u);
             };
             auto issue_pv = [&](int i, int st, bool acc) {
-                const uint64_t vd = sdesc_sw128(smem_u32(sV + st * C::KV_BYTES), BK * 128, 1024);
+                const uint32_t vd = sdesc_lo(smem_u32(sV + st * C::KV_BYTES), BK * 128);
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
-                    umma_ts(tmem + C::O_COL(i), tmem + C::S_COL(i) + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
-                            (acc || kk > 0) ? 1u : 0u);
+                    umma_ts_lo(tmem + C::O_COL(i), tmem + C::S_COL(i) + kk * 8, vd + ((kk * 16 * 128) >> 4), idesc_pv,
+                               (acc || kk > 0) ? 1u : 0u);
             };
             uint32_t kv_it = 0, q_it = 0, p_it[NQ] = {};
             bool ok = true;
