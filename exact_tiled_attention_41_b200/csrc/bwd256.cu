@@ -116,19 +116,27 @@ struct Cfg {
                               OFF_STAT = OFF_DS + 128 * 128,            // [2][-LSE2 x 64 | -Delta x 64]
                               OFF_BAR = OFF_STAT + 2 * 128 * 4;
     // kv_full, kv_empty | slot_full[NSLOT] | slot_empty[NSLOT] | stat_full[2] | stat_empty[2] |
-    // s_full, p_full, dq_full, dq_empty, dkv_full | unit feed
+    // s_full, p_full, dq_full, dq_empty, dkv_full, dk_done, dv_done | unit feed
     static constexpr int BAR_SLOT_FULL = 2, BAR_SLOT_EMPTY = 2 + NSLOT, BAR_STAT_FULL = 2 + 2 * NSLOT,
-                         BAR_STAT_EMPTY = BAR_STAT_FULL + 2, BAR_S_FULL = BAR_STAT_EMPTY + 2, BAR_FEED = BAR_S_FULL + 5;
+                         BAR_STAT_EMPTY = BAR_STAT_FULL + 2, BAR_S_FULL = BAR_STAT_EMPTY + 2, BAR_FEED = BAR_S_FULL + 7;
     static constexpr int NUM_BARS = BAR_FEED + 2 * kFeedSlots;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
     static_assert(SMEM <= 232448, "shared memory per block");
     static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
-    static constexpr int THREADS = 384, LAUNCH_REGS = 168, COMPUTE_REGS = 232, OTHER_REGS = 136;
-    static_assert(128 * COMPUTE_REGS + 2 * 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
+    // 16 warps: 0-7 two compute warpgroups (query columns 0-31 / 32-63), 8-11 dQ warpgroup, 12 producer,
+    // 13 and 14 the two MMA issuers, 15 idle.  Registers: launch at 128 per thread (512 x 128 = 65536); the
+    // producer / issuer warpgroup gives 40 per thread to the dQ warpgroup.  The host checks the launch count.
+    static constexpr int THREADS = 512, LAUNCH_REGS = 128, COMPUTE_REGS = 128, DQ_REGS = 168, OTHER_REGS = 88;
+    static_assert(2 * 128 * COMPUTE_REGS + 128 * DQ_REGS + 128 * OTHER_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
+// One issuing thread takes about 54 cycles per 16-deep MMA, more than the tensor core needs for the 128 x 64
+// products here, so two threads issue: A takes S^T, dQ^T and dK (the Q pairs are its operands), B takes dP^T
+// and dV (the dO pairs).  Each releases the ring slots of its own pairs.  S^T of a tile overwrites the P^T
+// that B's dV of the previous tile reads, and dP^T overwrites the dS^T that A's dK reads, so each issuer
+// waits for the other's previous product there (dv_done, dk_done).
 template <bool DQ>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ B256Params p) {
@@ -147,9 +155,9 @@ __global__ void __launch_bounds__(384, 1)
     auto stat_full = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_FULL + s); };
     auto stat_empty = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_EMPTY + s); };
     const uint32_t s_full = b0 + 8u * C::BAR_S_FULL, p_full = s_full + 8, dq_full = s_full + 16,
-                   dq_empty = s_full + 24, dkv_full = s_full + 32;
+                   dq_empty = s_full + 24, dkv_full = s_full + 32, dk_done = s_full + 40, dv_done = s_full + 48;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int PRODUCER = 8, MMA = 9;
+    constexpr int PRODUCER = 12, MMA_A = 13, MMA_B = 14;
 
     if ((smem_u32(smem) & 1023u) != 0) {
         if (threadIdx.x == 0) atomicCAS(p.status, 0, 2);
@@ -157,23 +165,25 @@ __global__ void __launch_bounds__(384, 1)
     }
     if (threadIdx.x == 0) {
         mbar_init(bars + 0, 1);                                      // kv_full
-        mbar_init(bars + 1, 1);                                      // kv_empty
+        mbar_init(bars + 1, 2);                                      // kv_empty: both issuers
         for (int s = 0; s < static_cast<int>(C::NSLOT); ++s) {
             mbar_init(bars + C::BAR_SLOT_FULL + s, 1);               // expect-tx arrival of the pair's loads
             mbar_init(bars + C::BAR_SLOT_EMPTY + s, 1);              // commit of the pair's last reader
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(bars + C::BAR_STAT_FULL + s, 32);              // the producer's 32 lanes
-            mbar_init(bars + C::BAR_STAT_EMPTY + s, 4);              // one arrival per compute warp
+            mbar_init(bars + C::BAR_STAT_EMPTY + s, 8);              // one arrival per compute warp
         }
-        mbar_init(bars + C::BAR_S_FULL + 0, 1);                      // s_full
-        mbar_init(bars + C::BAR_S_FULL + 1, 128);                    // p_full
+        mbar_init(bars + C::BAR_S_FULL + 0, 2);                      // s_full: S^T (A) and dP^T (B)
+        mbar_init(bars + C::BAR_S_FULL + 1, 256);                    // p_full: both compute warpgroups
         mbar_init(bars + C::BAR_S_FULL + 2, 1);                      // dq_full
         mbar_init(bars + C::BAR_S_FULL + 3, 128);                    // dq_empty
-        mbar_init(bars + C::BAR_S_FULL + 4, 1);                      // dkv_full
+        mbar_init(bars + C::BAR_S_FULL + 4, 2);                      // dkv_full: last dK (A) and dV (B)
+        mbar_init(bars + C::BAR_S_FULL + 5, 1);                      // dk_done
+        mbar_init(bars + C::BAR_S_FULL + 6, 1);                      // dv_done
         for (int s = 0; s < kFeedSlots; ++s) {
             mbar_init(bars + C::BAR_FEED + s, 1);                              // unit published
-            mbar_init(bars + C::BAR_FEED + kFeedSlots + s, DQ ? 9 : 5);        // read by MMA, compute (, dQ) warps
+            mbar_init(bars + C::BAR_FEED + kFeedSlots + s, DQ ? 14 : 10);      // read by the issuers, compute (, dQ) warps
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -184,7 +194,7 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_map(&tmV);
         tma_prefetch_map(&tmDO);
     }
-    if (warp == MMA) {
+    if (warp == MMA_A) {
         tmem_alloc(smem_u32(tmem_slot), 512);
         tmem_relinquish();
     }
@@ -195,7 +205,7 @@ __global__ void __launch_bounds__(384, 1)
     const Watch w{abort_flag, p.status, p.timeout_ns};
     const int G = p.group;
 
-    if (warp >= 4) {
+    if (warp >= 12) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
         if (warp == PRODUCER) {
             uint32_t unit_it = 0, q_it = 0;
@@ -270,21 +280,26 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             __syncwarp();
-        } else if (warp == MMA) {
+        } else if (warp == MMA_A || warp == MMA_B) {
             if (lane == 0) {
+                const bool isA = warp == MMA_A;
                 constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);     // S^T, dP^T
                 constexpr uint32_t id_g = idesc_bf16_f32(128, 128, false, true);     // dV, dK halves
                 constexpr uint32_t id_q = idesc_bf16_f32(128, 64, true, true);       // dQ^T half
-                // Descriptor low words, advanced by constant offsets >> 4 (one add per operand per MMA: the
-                // issuing thread needs about as long per MMA as the tensor core at N = 64, so the loop is kept
-                // free of any other arithmetic)
+                // Descriptor low words, advanced by constant offsets >> 4 (one add per operand per MMA)
                 constexpr uint32_t CHUNK16 = (128 * 128) >> 4, BOX16 = C::BOX_BYTES >> 4, PAIR16 = C::PAIR_BYTES >> 4,
                                    K16 = 32 >> 4, ROWS16 = (16 * 128) >> 4;
-                const uint32_t dK0 = sdesc_lo(smem_u32(smem + C::OFF_K), 16);           // K, K-major boxes
-                const uint32_t dV0 = sdesc_lo(smem_u32(smem + C::OFF_V), 16);           // V
+                // A: K and the Q pairs; B: V and the dO pairs
+                const uint32_t dKV = sdesc_lo(smem_u32(smem + (isA ? C::OFF_K : C::OFF_V)), 16);
                 const uint32_t dDS = sdesc_lo(smem_u32(smem + C::OFF_DS), 128 * 128);   // dS^T, dQ^T's B (MN-major)
                 const uint32_t dRK = sdesc_lo(smem_u32(smem + C::OFF_RING), 16);        // ring pairs, K-major
                 const uint32_t dRN = sdesc_lo(smem_u32(smem + C::OFF_RING), C::BOX_BYTES);   // ring pairs, MN-major
+                // this issuer's pairs of a tile: A reads Q other (0) and Q own (2); B reads dO other (1), dO own (3)
+                const uint32_t k_other = isA ? 0u : 1u, k_own = isA ? 2u : 3u;
+                const uint32_t col_s = isA ? C::COL_S : C::COL_DP;                     // S^T or dP^T
+                const uint32_t col_g = isA ? C::COL_DK : C::COL_DV;                    // dK or dV
+                const uint32_t col_a = isA ? C::COL_DP : C::COL_S;                     // dS^T or P^T (A operand)
+                const uint32_t done_mine = isA ? dk_done : dv_done, done_other = isA ? dv_done : dk_done;
                 uint32_t unit_it = 0, q_it = 0;
                 bool ok = true;
                 for (uint32_t fi = 0; ok; ++fi) {
@@ -295,80 +310,54 @@ __global__ void __launch_bounds__(384, 1)
                     if (t.skip || t.n_it == 0) continue;
                     if (!mbar_wait(kv_full, unit_it & 1, w)) { ok = false; break; }
                     const int oh = 1 - t.hh;
-                    const uint32_t kO = dK0 + 2 * oh * CHUNK16, kH = dK0 + 2 * t.hh * CHUNK16;
-                    const uint32_t vO = dV0 + 2 * oh * CHUNK16, vH = dV0 + 2 * t.hh * CHUNK16;
+                    const uint32_t xO = dKV + 2 * oh * CHUNK16, xH = dKV + 2 * t.hh * CHUNK16;
                     // K[:, half]^T as dQ^T's A operand (MN-major: the two 64-column boxes of the half, 16 KB apart)
                     const uint32_t kT = sdesc_lo(smem_u32(smem + C::OFF_K + 2 * t.hh * 128 * 128), 128 * 128);
                     for (int it = 0; it < t.n_it; ++it, ++q_it) {
-                        // ring slots of the tile's pairs: Q other half, dO other half, Q own half, dO own half
                         const uint32_t px = 4u * q_it;
-                        uint32_t sl[4];
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) sl[k] = (px + k) % C::NSLOT;
-                        auto pair_ready = [&](int k) {
-                            return mbar_wait(slot_full(sl[k]), ((px + k) / C::NSLOT) & 1, w);
-                        };
-                        const uint32_t q0 = dRK + sl[0] * PAIR16, o1 = dRK + sl[1] * PAIR16,
-                                       q2 = dRK + sl[2] * PAIR16, o3 = dRK + sl[3] * PAIR16;
-                        const uint32_t q2n = dRN + sl[2] * PAIR16, o3n = dRN + sl[3] * PAIR16;
-                        if (!pair_ready(0) || !pair_ready(2)) { ok = false; break; }
+                        const uint32_t slo = (px + k_other) % C::NSLOT, sho = (px + k_own) % C::NSLOT;
+                        const uint32_t po = dRK + slo * PAIR16, ph = dRK + sho * PAIR16, phn = dRN + sho * PAIR16;
+                        if (!mbar_wait(slot_full(slo), ((px + k_other) / C::NSLOT) & 1, w)) { ok = false; break; }
+                        // the other issuer's product of the previous tile has read what this one overwrites
+                        if (q_it > 0 && !mbar_wait(done_other, (q_it - 1) & 1, w)) { ok = false; break; }
+                        if (isA && !mbar_wait(slot_full(sho), ((px + k_own) / C::NSLOT) & 1, w)) { ok = false; break; }
                         tc_fence_after();
-                        // S^T = K Q^T over the head dim, the other half's chunks first
+                        // S^T = K Q^T (A) or dP^T = V dO^T (B) over the head dim, the other half's chunks first
 #pragma unroll
                         for (int i = 0; i < 2; ++i)
 #pragma unroll
                             for (int k4 = 0; k4 < 4; ++k4)
-                                umma_ss_lo(tmem + C::COL_S, kO + i * CHUNK16 + k4 * K16, q0 + i * BOX16 + k4 * K16, id_s,
+                                umma_ss_lo(tmem + col_s, xO + i * CHUNK16 + k4 * K16, po + i * BOX16 + k4 * K16, id_s,
                                            (i | k4) != 0);
+                        if (!isA) {
+                            umma_commit(slot_empty(slo));         // dO of the other half: last read by dP^T
+                            if (!mbar_wait(slot_full(sho), ((px + k_own) / C::NSLOT) & 1, w)) { ok = false; break; }
+                            tc_fence_after();
+                        }
 #pragma unroll
                         for (int i = 0; i < 2; ++i)
 #pragma unroll
                             for (int k4 = 0; k4 < 4; ++k4)
-                                umma_ss_lo(tmem + C::COL_S, kH + i * CHUNK16 + k4 * K16, q2 + i * BOX16 + k4 * K16, id_s,
-                                           1u);
-                        umma_commit(slot_empty(sl[0]));           // Q of the other half: last read by S^T
-                        if (!pair_ready(1)) { ok = false; break; }
-                        tc_fence_after();
-                        // dP^T = V dO^T, the other half first (its pair is loaded early), then the own half
-#pragma unroll
-                        for (int i = 0; i < 2; ++i)
-#pragma unroll
-                            for (int k4 = 0; k4 < 4; ++k4)
-                                umma_ss_lo(tmem + C::COL_DP, vO + i * CHUNK16 + k4 * K16, o1 + i * BOX16 + k4 * K16, id_s,
-                                           (i | k4) != 0);
-                        umma_commit(slot_empty(sl[1]));           // dO of the other half: last read by dP^T
-                        if (!pair_ready(3)) { ok = false; break; }
-                        tc_fence_after();
-#pragma unroll
-                        for (int i = 0; i < 2; ++i)
-#pragma unroll
-                            for (int k4 = 0; k4 < 4; ++k4)
-                                umma_ss_lo(tmem + C::COL_DP, vH + i * CHUNK16 + k4 * K16, o3 + i * BOX16 + k4 * K16, id_s,
-                                           1u);
+                                umma_ss_lo(tmem + col_s, xH + i * CHUNK16 + k4 * K16, ph + i * BOX16 + k4 * K16, id_s, 1u);
+                        if (isA) umma_commit(slot_empty(slo));    // Q of the other half: last read by S^T
                         umma_commit(s_full);
                         if (!mbar_wait(p_full, q_it & 1, w)) { ok = false; break; }
-                        if (DQ && q_it > 0 && !mbar_wait(dq_empty, (q_it - 1) & 1, w)) { ok = false; break; }
+                        if (DQ && isA && q_it > 0 && !mbar_wait(dq_empty, (q_it - 1) & 1, w)) { ok = false; break; }
                         tc_fence_after();
-                        if constexpr (DQ) {
+                        if (DQ && isA) {
                             // dQ^T half = K[:, half]^T dS^T (K-dim = 128 keys)
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)
                                 umma_ss_lo(tmem + C::COL_DQ, kT + kk * ROWS16, dDS + kk * ROWS16, id_q, kk > 0);
                             umma_commit(dq_full);
                         }
-                        // dK half += dS^T Q[:, half], then dV half += P^T dO[:, half] (K-dim = 64 queries): the
-                        // own-half Q pair is released first, because the next tile's last pair waits for its slot
+                        // dK half += dS^T Q[:, half] (A) or dV half += P^T dO[:, half] (B), K-dim = 64 queries
                         const uint32_t first = it > 0 ? 1u : 0u;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_ts_lo(tmem + C::COL_DK, tmem + C::COL_DP + kk * 8, q2n + kk * ROWS16, id_g,
-                                       kk > 0 ? 1u : first);
-                        umma_commit(slot_empty(sl[2]));
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_ts_lo(tmem + C::COL_DV, tmem + C::COL_S + kk * 8, o3n + kk * ROWS16, id_g,
-                                       kk > 0 ? 1u : first);
-                        umma_commit(slot_empty(sl[3]));
+                            umma_ts_lo(tmem + col_g, tmem + col_a + kk * 8, phn + kk * ROWS16, id_g, kk > 0 ? 1u : first);
+                        umma_commit(slot_empty(sho));             // the own-half pair: last read here
+                        umma_commit(done_mine);
                     }
                     if (!ok) break;
                     umma_commit(dkv_full);
@@ -377,9 +366,12 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             __syncwarp();
-        } else if (DQ && warp < 8) {
+        }
+    } else if (warp >= 8) {
+        if constexpr (DQ) {
+            asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::DQ_REGS));
             // -------------------------------------------------------- dQ warpgroup (thread = head-dim row)
-            const int wq = warp - 4;
+            const int wq = warp - 8;
             const uint32_t lb = tmem_lane_base(wq);
             uint32_t q_it = 0;
             bool ok = true;
@@ -450,10 +442,10 @@ __global__ void __launch_bounds__(384, 1)
             }
         }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::COMPUTE_REGS));
-        // ------------------------------------------------------------ compute warpgroup (thread = key row)
-        const int r = warp * 32 + lane;
-        const uint32_t lb = tmem_lane_base(warp);
+        // ------------------------------------------------------------ compute warpgroups (thread = key row)
+        const int gq = warp >> 2;                  // query columns [32 gq, 32 gq + 32)
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lb = tmem_lane_base(warp & 3);
         const float c2 = p.scale_log2;
         uint32_t unit_it = 0, q_it = 0;
         bool ok = true;
@@ -466,13 +458,12 @@ __global__ void __launch_bounds__(384, 1)
             const int kj = t.n0 + r;
             const bool kvalid = kj < t.Lk;
             const size_t krow = (static_cast<size_t>(t.k_start) + kj) * p.Hkv + t.hk;
+            // warpgroup 0 owns dV of the unit's half, warpgroup 1 dK
+            __nv_bfloat16* dst = (gq == 0 ? p.dv : p.dk) + krow * D + t.hh * 128;
             if (t.n_it == 0) {
                 if (kvalid) {
                     const uint4 z = make_uint4(0, 0, 0, 0);
-                    for (int c = 0; c < 16; ++c) {
-                        reinterpret_cast<uint4*>(p.dk + krow * D + t.hh * 128)[c] = z;
-                        reinterpret_cast<uint4*>(p.dv + krow * D + t.hh * 128)[c] = z;
-                    }
+                    for (int c = 0; c < 16; ++c) reinterpret_cast<uint4*>(dst)[c] = z;
                 }
                 continue;
             }
@@ -485,48 +476,40 @@ __global__ void __launch_bounds__(384, 1)
                 if (!mbar_wait(s_full, q_it & 1, w)) { ok = false; break; }
                 const uint32_t sb = q_it & 1;
                 if (!mbar_wait(stat_full(sb), (q_it >> 1) & 1, w)) { ok = false; break; }
-                const float* nL = sStat + sb * 128;      // -LSE2 of the tile's 64 rows
-                const float* nD = nL + 64;               // -Delta
+                const float* nL = sStat + sb * 128 + 32 * gq;      // -LSE2 of this warpgroup's 32 rows
+                const float* nD = nL + 64;                         // -Delta
                 tc_fence_after();
-                uint32_t sa[2][32], da[2][32];
-                tmem_ld32(tmem + lb + C::COL_S, sa[0]);
-                tmem_ld32(tmem + lb + C::COL_S + 32, sa[1]);
-                tmem_ld32(tmem + lb + C::COL_DP, da[0]);
-                tmem_ld32(tmem + lb + C::COL_DP + 32, da[1]);
-                tmem_ld_wait_tie(sa[0]);
-                reg_tie(sa[1]);
-                reg_tie(da[0]);
-                reg_tie(da[1]);
-                const int qmin = q_lo - m0, qmax = q_hi - m0;
-                const bool any_mask = __any_sync(0xffffffffu, !(kvalid && qmin <= 0 && qmax >= 63));
+                uint32_t sa[32], da[32];
+                tmem_ld32(tmem + lb + C::COL_S + 32 * gq, sa);
+                tmem_ld32(tmem + lb + C::COL_DP + 32 * gq, da);
+                tmem_ld_wait_tie(sa);
+                reg_tie(da);
+                const int qmin = q_lo - m0 - 32 * gq, qmax = q_hi - m0 - 32 * gq;
+                const bool any_mask = __any_sync(0xffffffffu, !(kvalid && qmin <= 0 && qmax >= 31));
                 const float2 c2v = make_float2(c2, c2);
+                uint32_t pp[16], dd[16];
+#pragma unroll
+                for (int e = 0; e < 32; e += 2) {
+                    const float2 sv = make_float2(__uint_as_float(sa[e]), __uint_as_float(sa[e + 1]));
+                    const float2 dv = make_float2(__uint_as_float(da[e]), __uint_as_float(da[e + 1]));
+                    const float2 a = ffma2(sv, c2v, make_float2(nL[e], nL[e + 1]));
+                    float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
+                    if (any_mask) {
+                        pr.x = (kvalid && e >= qmin && e <= qmax) ? pr.x : 0.f;
+                        pr.y = (kvalid && e + 1 >= qmin && e + 1 <= qmax) ? pr.y : 0.f;
+                    }
+                    const float2 ds = fmul2(pr, fadd2(dv, make_float2(nD[e], nD[e + 1])));
+                    pp[e / 2] = pack_bf16x2(pr.x, pr.y);
+                    dd[e / 2] = pack_bf16x2(ds.x, ds.y);
+                }
+                tmem_st16(tmem + lb + C::COL_S + 16 * gq, pp);
+                tmem_st16(tmem + lb + C::COL_DP + 16 * gq, dd);
                 uint8_t* ds_row = smem + C::OFF_DS + r * 128;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t pp[16], dd[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int qc = half * 32 + e;
-                        const float2 sv = make_float2(__uint_as_float(sa[half][e]), __uint_as_float(sa[half][e + 1]));
-                        const float2 dv = make_float2(__uint_as_float(da[half][e]), __uint_as_float(da[half][e + 1]));
-                        const float2 a = ffma2(sv, c2v, make_float2(nL[qc], nL[qc + 1]));
-                        float2 pr = make_float2(ex2_approx(a.x), ex2_approx(a.y));
-                        if (any_mask) {
-                            pr.x = (kvalid && qc >= qmin && qc <= qmax) ? pr.x : 0.f;
-                            pr.y = (kvalid && qc + 1 >= qmin && qc + 1 <= qmax) ? pr.y : 0.f;
-                        }
-                        const float2 ds = fmul2(pr, fadd2(dv, make_float2(nD[qc], nD[qc + 1])));
-                        pp[e / 2] = pack_bf16x2(pr.x, pr.y);
-                        dd[e / 2] = pack_bf16x2(ds.x, ds.y);
-                    }
-                    tmem_st16(tmem + lb + C::COL_S + 16 * half, pp);
-                    tmem_st16(tmem + lb + C::COL_DP + 16 * half, dd);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int cin = half * 4 + q4;
-                        *reinterpret_cast<uint4*>(ds_row + ((cin ^ (r & 7)) << 4)) =
-                            make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
-                    }
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int cin = gq * 4 + q4;
+                    *reinterpret_cast<uint4*>(ds_row + ((cin ^ (r & 7)) << 4)) =
+                        make_uint4(dd[4 * q4], dd[4 * q4 + 1], dd[4 * q4 + 2], dd[4 * q4 + 3]);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(stat_empty(sb));   // the warp has read the tile's statistics
@@ -539,29 +522,23 @@ __global__ void __launch_bounds__(384, 1)
             if (!mbar_wait(dkv_full, unit_it & 1, w)) { ok = false; break; }
             ++unit_it;
             tc_fence_after();
+            const uint32_t col = gq == 0 ? C::COL_DV : C::COL_DK;
+            const float2 mul2 = gq == 0 ? make_float2(1.f, 1.f) : make_float2(p.scale, p.scale);
 #pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col = which == 0 ? C::COL_DV : C::COL_DK;
-                const float2 mul2 = which == 0 ? make_float2(1.f, 1.f) : make_float2(p.scale, p.scale);
-                __nv_bfloat16* dst = (which == 0 ? p.dv : p.dk) + krow * D + t.hh * 128;
-#pragma unroll 1
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t ra[32];
-                    tmem_ld32(tmem + lb + col + cc * 32, ra);
-                    tmem_ld_wait_tie(ra);
-                    uint32_t pk[16];
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t ra[32];
+                tmem_ld32(tmem + lb + col + cc * 32, ra);
+                tmem_ld_wait_tie(ra);
+                uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float2 v =
-                            fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), mul2);
-                        pk[e] = pack_bf16x2(v.x, v.y);
-                    }
-                    if (kvalid) {
-                        uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
+                for (int e = 0; e < 16; ++e) {
+                    const float2 v = fmul2(make_float2(__uint_as_float(ra[2 * e]), __uint_as_float(ra[2 * e + 1])), mul2);
+                    pk[e] = pack_bf16x2(v.x, v.y);
+                }
+                if (kvalid) {
+                    uint4* o4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
-                    }
+                    for (int e = 0; e < 4; ++e) o4[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
                 }
             }
             tc_fence_before();
@@ -574,7 +551,7 @@ __global__ void __launch_bounds__(384, 1)
         while (global_timer_ns() - t0 < 200000ull) {
         }
     }
-    if (warp == MMA) {
+    if (warp == MMA_A) {
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
