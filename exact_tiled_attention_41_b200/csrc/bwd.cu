@@ -140,7 +140,7 @@ struct BwdCfg {
     static constexpr uint32_t OFF_K = 0, OFF_V = T_BYTES, OFF_Q = 2 * T_BYTES, OFF_DO = (2 + ST) * T_BYTES,
                               OFF_DS = (2 + 2 * ST) * T_BYTES, OFF_STAT = OFF_DS + DS_BYTES,
                               OFF_BAR = OFF_STAT + 2 * ST * 128 * 4;
-    static constexpr int NUM_BARS = 2 + 2 * ST + 9 + 2 * kFeedSlots;
+    static constexpr int NUM_BARS = 2 + 2 * ST + 10 + 2 * kFeedSlots;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
     // tensor memory: dV | dK | S^T | dP^T.  After the gradient step the packed bf16 P^T and dS^T of each
     // 32-query half sit in that half's own 32 columns of S^T; dQ (fp32, D columns) is accumulated over
@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(512, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
     int* feed_slot = reinterpret_cast<int*>(tmem_slot + 4);
     const uint32_t b0 = smem_u32(bars);
-    const UnitFeed feed{feed_slot, b0 + 8u * (2 + 2 * ST + 9), b0 + 8u * (2 + 2 * ST + 9 + kFeedSlots)};
+    const UnitFeed feed{feed_slot, b0 + 8u * (2 + 2 * ST + 10), b0 + 8u * (2 + 2 * ST + 10 + kFeedSlots)};
     // K and V of a unit arrive / are released separately: V is last read by the unit's last dP^T,
     // K by its last dQ (or S^T), so the next unit's V and first Q/dO tile load while those finish
     const uint32_t k_full = b0, k_free = b0 + 8;
@@ -186,10 +186,10 @@ __global__ void __launch_bounds__(512, 1)
     // p_full / p_full_hi: compute warpgroup 0 (query columns 0-63) / 1 (64-127) done
     const uint32_t s_full = b0 + 8u * (2 + 2 * ST), p_full = s_full + 8, dq_full = s_full + 16,
                    dq_empty = s_full + 24, dkv_full = s_full + 32, dq_empty_hi = s_full + 40, p_full_hi = s_full + 48,
-                   v_full = s_full + 56, v_free = s_full + 64;
+                   v_full = s_full + 56, v_free = s_full + 64, dv_done = s_full + 72;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr int PRODUCER = 12, MMA = 13;
+    constexpr int PRODUCER = 12, MMA = 13, MMA_B = 14;
 
     if ((smem_u32(smem) & 1023u) != 0) {   // the swizzled tiles need a 1024-byte aligned base
         if (threadIdx.x == 0) atomicCAS(p.status, 0, 2);
@@ -200,20 +200,21 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bars + 1, 1);
         for (int s = 0; s < ST; ++s) {
             mbar_init(bars + 2 + s, 33);        // 32 producer lanes (statistics) + the TMA expect-tx arrival
-            mbar_init(bars + 2 + ST + s, 1);
+            mbar_init(bars + 2 + ST + s, 2);    // both issuers' last reads of the stage
         }
-        mbar_init(bars + 2 + 2 * ST + 0, 1);    // s_full
+        mbar_init(bars + 2 + 2 * ST + 0, 2);    // s_full: S^T (issuer A) and dP^T (issuer B)
         mbar_init(bars + 2 + 2 * ST + 1, 128);  // p_full: compute warpgroup 0 (query columns 0-63)
         mbar_init(bars + 2 + 2 * ST + 2, 1);    // dq_full
         mbar_init(bars + 2 + 2 * ST + 3, 128);  // dq_empty: dQ columns in the S^T region read out
-        mbar_init(bars + 2 + 2 * ST + 4, 1);    // dkv_full
+        mbar_init(bars + 2 + 2 * ST + 4, 2);    // dkv_full: last dK (A) and dV (B)
         mbar_init(bars + 2 + 2 * ST + 5, 128);  // dq_empty_hi: dQ columns in the dP^T region read out
         mbar_init(bars + 2 + 2 * ST + 6, 128);  // p_full_hi: compute warpgroup 1 (query columns 64-127)
         mbar_init(bars + 2 + 2 * ST + 7, 1);    // v_full
         mbar_init(bars + 2 + 2 * ST + 8, 1);    // v_free
+        mbar_init(bars + 2 + 2 * ST + 9, 1);    // dv_done: issuer B's dV of a tile has read P^T
         for (int s = 0; s < kFeedSlots; ++s) {
-            mbar_init(bars + 2 + 2 * ST + 9 + s, 1);                             // unit published
-            mbar_init(bars + 2 + 2 * ST + 9 + kFeedSlots + s, DQ ? 13 : 9);      // read by MMA, compute (, dQ) warps
+            mbar_init(bars + 2 + 2 * ST + 10 + s, 1);                            // unit published
+            mbar_init(bars + 2 + 2 * ST + 10 + kFeedSlots + s, DQ ? 14 : 10);    // read by the issuers, compute (, dQ) warps
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -304,24 +305,29 @@ __global__ void __launch_bounds__(512, 1)
                     if (!load_tile(it)) ok = false;
             }
             __syncwarp();
-        } else if (warp == MMA) {
-            // -------------------------------------------------------- MMA issuer
+        } else if (warp == MMA || warp == MMA_B) {
+            // -------------------------------------------------------- MMA issuers
+            // One issuing thread needs about 54 cycles per 16-deep MMA, close to the 64 the tensor core
+            // needs for these 128 x 128 steps, so the waits between products leave the tensor core idle.  Two
+            // threads issue: A takes S^T, dK and dQ (K and Q are its operands), B takes dP^T and dV (V, dO).
+            // S^T of a tile overwrites the packed P^T that B's dV of the previous tile reads (dv_done); dP^T
+            // overwrites the previous dQ, read out by the dQ warpgroup (dq_empty).
             if (lane == 0) {
+                const bool isA = warp == MMA;
                 constexpr uint32_t id_kk = idesc_bf16_f32(128, 128, false, false);   // S^T, dP^T
                 constexpr uint32_t id_tn = idesc_bf16_f32(128, D, false, true);      // dV, dK (A in tensor memory)
                 constexpr uint32_t id_dq = idesc_bf16_f32(128, D, true, true);       // dQ, all D columns
-                // Descriptor low words, advanced by constant offsets >> 4: one add per operand per MMA, so the
-                // issuing thread keeps up with the tensor core (about 54 cycles per MMA at best from one
-                // thread, against 64 for these 128 x 128 x 16 steps)
+                // Descriptor low words, advanced by constant offsets >> 4 (one add per operand per MMA)
                 constexpr uint32_t T16 = C::T_BYTES >> 4, ROWS16 = (16 * 128) >> 4;
-                const uint32_t dK0 = sdesc_lo(smem_u32(smem + C::OFF_K), 16);             // K, K-major
-                const uint32_t dV0 = sdesc_lo(smem_u32(smem + C::OFF_V), 16);             // V, K-major
-                const uint32_t dQ0 = sdesc_lo(smem_u32(smem + C::OFF_Q), 16);             // Q stage 0, K-major
-                const uint32_t dO0 = sdesc_lo(smem_u32(smem + C::OFF_DO), 16);            // dO stage 0, K-major
-                const uint32_t dQ0n = sdesc_lo(smem_u32(smem + C::OFF_Q), 128 * 128);     // Q as MN-major B
-                const uint32_t dO0n = sdesc_lo(smem_u32(smem + C::OFF_DO), 128 * 128);    // dO as MN-major B
+                // A: K and Q; B: V and dO
+                const uint32_t dX0 = sdesc_lo(smem_u32(smem + (isA ? C::OFF_K : C::OFF_V)), 16);      // K-major
+                const uint32_t dY0 = sdesc_lo(smem_u32(smem + (isA ? C::OFF_Q : C::OFF_DO)), 16);     // stage 0, K-major
+                const uint32_t dY0n = sdesc_lo(smem_u32(smem + (isA ? C::OFF_Q : C::OFF_DO)), 128 * 128);   // MN-major B
                 const uint32_t dSn = sdesc_lo(smem_u32(smem + C::OFF_DS), 128 * 128);     // dS, MN-major A of dQ
                 const uint32_t dKn = sdesc_lo(smem_u32(smem + C::OFF_K), 128 * 128);      // K, MN-major B of dQ
+                const uint32_t col_s = isA ? C::COL_S : C::COL_DP;                         // S^T or dP^T
+                const uint32_t col_g = isA ? C::COL_DK : C::COL_DV;                        // dK or dV
+                const uint32_t a_off = isA ? 16u : 0u;                                     // packed dS^T / P^T
                 auto kchunk = [](int kk) { return static_cast<uint32_t>(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4); };
                 uint32_t unit_it = 0, q_it = 0, g_it = 0;
                 bool ok = true;
@@ -331,40 +337,38 @@ __global__ void __launch_bounds__(512, 1)
                     if (u < 0) break;
                     const BUnit t = decode_bunit(p, u);
                     if (t.skip || t.n_it == 0) continue;
-                    if (!mbar_wait(k_full, unit_it & 1, w)) { ok = false; break; }
-                    if (!mbar_wait(v_full, unit_it & 1, w)) { ok = false; break; }
+                    if (!mbar_wait(isA ? k_full : v_full, unit_it & 1, w)) { ok = false; break; }
                     for (int it = 0; it < t.n_it; ++it, ++q_it, ++g_it) {
                         const bool last = it + 1 == t.n_it;
                         const int st = q_it % ST;
                         if (!mbar_wait(q_full(st), (q_it / ST) & 1, w)) { ok = false; break; }
+                        if (isA) {
+                            // S^T overwrites the packed P^T that the previous tile's dV read
+                            if (g_it > 0 && !mbar_wait(dv_done, (g_it - 1) & 1, w)) { ok = false; break; }
+                        } else if (DQ && g_it > 0) {
+                            // dP^T goes where the previous tile's dQ was: both halves of it must be read out
+                            if (!mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
+                            if (!mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
+                        }
                         tc_fence_after();
-                        const uint32_t qd = dQ0 + st * T16, od = dO0 + st * T16;
-                        const uint32_t qn = dQ0n + st * T16, on = dO0n + st * T16;
+                        const uint32_t yd = dY0 + st * T16, yn = dY0n + st * T16;
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk)
-                            umma_ss_lo(tmem + C::COL_S, dK0 + kchunk(kk), qd + kchunk(kk), id_kk, kk > 0);
-                        if (!DQ && last) umma_commit(k_free);     // K's last reader without the dQ product
-                        // dP^T goes where the previous tile's dQ was: both halves of it must be read out
-                        if (DQ && g_it > 0 && !mbar_wait(dq_empty, (g_it - 1) & 1, w)) { ok = false; break; }
-                        if (DQ && g_it > 0 && !mbar_wait(dq_empty_hi, (g_it - 1) & 1, w)) { ok = false; break; }
-                        tc_fence_after();
-#pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk)
-                            umma_ss_lo(tmem + C::COL_DP, dV0 + kchunk(kk), od + kchunk(kk), id_kk, kk > 0);
+                            umma_ss_lo(tmem + col_s, dX0 + kchunk(kk), yd + kchunk(kk), id_kk, kk > 0);
                         umma_commit(s_full);
-                        if (last) umma_commit(v_free);            // V's last reader in this unit
-                        // dV += P^T dO, dK += dS^T Q over queries 0-63, as soon as warpgroup 0 is done
+                        if (isA && !DQ && last) umma_commit(k_free);   // K's last reader without the dQ product
+                        if (!isA && last) umma_commit(v_free);         // V's last reader in this unit
+                        // dK += dS^T Q (A) or dV += P^T dO (B) over queries 0-63, as soon as warpgroup 0 is done
                         if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t first = it > 0 ? 1u : 0u;
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            umma_ts_lo(tmem + C::COL_DV, tmem + C::COL_P(kk), on + kk * ROWS16, id_tn, kk > 0 ? 1u : first);
-                            umma_ts_lo(tmem + C::COL_DK, tmem + C::COL_DSP(kk), qn + kk * ROWS16, id_tn, kk > 0 ? 1u : first);
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_ts_lo(tmem + col_g, tmem + C::COL_P(kk) + a_off, yn + kk * ROWS16, id_tn,
+                                       kk > 0 ? 1u : first);
                         if (!mbar_wait(p_full_hi, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
-                        if constexpr (DQ) {
+                        if (DQ && isA) {
                             // dQ = dS K over dP^T's columns (read out by the dQ warpgroup while dV / dK finish)
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)     // K-dim = 128 key rows
@@ -372,13 +376,12 @@ __global__ void __launch_bounds__(512, 1)
                             umma_commit(dq_full);
                             if (last) umma_commit(k_free);        // K's last reader in this unit
                         }
-                        // dV, dK over queries 64-127
+                        // queries 64-127
 #pragma unroll
-                        for (int kk = 4; kk < 8; ++kk) {
-                            umma_ts_lo(tmem + C::COL_DV, tmem + C::COL_P(kk), on + kk * ROWS16, id_tn, 1u);
-                            umma_ts_lo(tmem + C::COL_DK, tmem + C::COL_DSP(kk), qn + kk * ROWS16, id_tn, 1u);
-                        }
+                        for (int kk = 4; kk < 8; ++kk)
+                            umma_ts_lo(tmem + col_g, tmem + C::COL_P(kk) + a_off, yn + kk * ROWS16, id_tn, 1u);
                         umma_commit(q_empty(st));
+                        if (!isA) umma_commit(dv_done);
                     }
                     if (!ok) break;
                     umma_commit(dkv_full);
