@@ -358,28 +358,24 @@ __global__ void __launch_bounds__(512, 1)
                         umma_commit(s_full);
                         if (isA && !DQ && last) umma_commit(k_free);   // K's last reader without the dQ product
                         if (!isA && last) umma_commit(v_free);         // V's last reader in this unit
-                        // dK += dS^T Q (A) or dV += P^T dO (B) over queries 0-63, as soon as warpgroup 0 is done
+                        // once both compute warpgroups are done: dQ first (A), so that its read-out, and with it
+                        // the next dP^T, starts early; then dK += dS^T Q (A) and dV += P^T dO (B)
                         if (!mbar_wait(p_full, g_it & 1, w)) { ok = false; break; }
-                        tc_fence_after();
-                        const uint32_t first = it > 0 ? 1u : 0u;
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_ts_lo(tmem + col_g, tmem + C::COL_P(kk) + a_off, yn + kk * ROWS16, id_tn,
-                                       kk > 0 ? 1u : first);
                         if (!mbar_wait(p_full_hi, g_it & 1, w)) { ok = false; break; }
                         tc_fence_after();
                         if (DQ && isA) {
-                            // dQ = dS K over dP^T's columns (read out by the dQ warpgroup while dV / dK finish)
+                            // dQ = dS K over dP^T's columns (read out by the dQ warpgroup while dV / dK run)
 #pragma unroll
                             for (int kk = 0; kk < 8; ++kk)     // K-dim = 128 key rows
                                 umma_ss_lo(tmem + C::COL_DQ, dSn + kk * ROWS16, dKn + kk * ROWS16, id_dq, kk > 0);
                             umma_commit(dq_full);
                             if (last) umma_commit(k_free);        // K's last reader in this unit
                         }
-                        // queries 64-127
+                        const uint32_t first = it > 0 ? 1u : 0u;
 #pragma unroll
-                        for (int kk = 4; kk < 8; ++kk)
-                            umma_ts_lo(tmem + col_g, tmem + C::COL_P(kk) + a_off, yn + kk * ROWS16, id_tn, 1u);
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_ts_lo(tmem + col_g, tmem + C::COL_P(kk) + a_off, yn + kk * ROWS16, id_tn,
+                                       kk > 0 ? 1u : first);
                         umma_commit(q_empty(st));
                         if (!isA) umma_commit(dv_done);
                     }
