@@ -235,6 +235,8 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t tmem = *tmem_slot;
     const Watch w{abort_flag, p.status, p.timeout_ns};
     const int G = p.group;
+    // the preprocess kernel's outputs (statistics, zeroed accumulator and unit counter) are read from here on
+    grid_dep_wait();
 
     if (warp >= 12) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::OTHER_REGS));
@@ -626,6 +628,7 @@ __global__ void __launch_bounds__(512, 1)
     }
 
     __syncthreads();
+    if (threadIdx.x == 0) grid_dep_launch();   // this CTA is done: the dQ convert may be scheduled
     if (*abort_flag) {
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 200000ull) {
@@ -1005,6 +1008,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
                                                       long long lse_sH, int lse_sT) {
     const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
+    // the main kernel may start its prologue now; it waits for this grid before reading anything written here
+    if (threadIdx.x == 0) grid_dep_launch();
     if (counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *counter = 0;
     const long long rows = static_cast<long long>(Tq) * Hq;
     if (dq_acc != nullptr) {
@@ -1053,31 +1058,33 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
 }
 
 // ---------------------------------------------------------------------------- convert
-// dQ[tok][h][:] = bf16(scale * dQacc[h][:/4][tok][:%4]); 32 tokens x D per block through shared memory.
+// dQ[tok][h][:] = bf16(scale * dQacc[h][:/4][tok][:%4]) for 32 tokens of one head per block: float4 columns
+// of 32 consecutive tokens are read (512 bytes per warp), staged in shared memory with one float4 of padding
+// per token row (each group of 8 lanes then writes 8 different bank groups), and leave as whole D-value rows
+// (D / 8 lanes x 16 bytes per token).  Launched after the main kernel with programmatic serialization: the
+// wait below covers the main kernel's last reduce-adds.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(const float* dq_acc, __nv_bfloat16* dq, int Tq, int Hq,
                                                           float scale) {
-    __shared__ float tile[32][D + 4];
+    constexpr int W4 = D / 4 + 1;                  // float4 per staged token row, with padding
+    __shared__ float4 tile[32 * W4];
+    grid_dep_wait();
     const int h = blockIdx.y;
     const int t0 = blockIdx.x * 32;
+    const float4* src = reinterpret_cast<const float4*>(dq_acc) + static_cast<size_t>(h) * (D / 4) * Tq + t0;
     for (int i = threadIdx.x; i < 32 * (D / 4); i += blockDim.x) {
         const int d4 = i / 32, tt = i % 32;
-        if (t0 + tt < Tq) {
-            const float4 v =
-                reinterpret_cast<const float4*>(dq_acc)[(static_cast<size_t>(h) * (D / 4) + d4) * Tq + t0 + tt];
-            tile[tt][4 * d4 + 0] = v.x;
-            tile[tt][4 * d4 + 1] = v.y;
-            tile[tt][4 * d4 + 2] = v.z;
-            tile[tt][4 * d4 + 3] = v.w;
-        }
+        if (t0 + tt < Tq) tile[tt * W4 + d4] = __ldcs(src + static_cast<size_t>(d4) * Tq + tt);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < 32 * (D / 2); i += blockDim.x) {
-        const int tt = i / (D / 2), d2 = i % (D / 2);
-        if (t0 + tt < Tq) {
-            const uint32_t v = pack_bf16x2(tile[tt][2 * d2] * scale, tile[tt][2 * d2 + 1] * scale);
-            reinterpret_cast<uint32_t*>(dq + (static_cast<size_t>(t0 + tt) * Hq + h) * D)[d2] = v;
-        }
+    constexpr int LPR = D / 8;                     // lanes per token row, 8 values (16 bytes) each
+    for (int i = threadIdx.x; i < 32 * LPR; i += blockDim.x) {
+        const int tt = i / LPR, c8 = i % LPR;
+        if (t0 + tt >= Tq) continue;
+        const float4 a = tile[tt * W4 + 2 * c8], b = tile[tt * W4 + 2 * c8 + 1];
+        const uint4 o = make_uint4(pack_bf16x2(a.x * scale, a.y * scale), pack_bf16x2(a.z * scale, a.w * scale),
+                                   pack_bf16x2(b.x * scale, b.y * scale), pack_bf16x2(b.z * scale, b.w * scale));
+        reinterpret_cast<uint4*>(dq + (static_cast<size_t>(t0 + tt) * Hq + h) * D)[c8] = o;
     }
 }
 
@@ -1186,14 +1193,17 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     const int grid = p.num_units < dev.num_sms ? p.num_units : dev.num_sms;
     if (grid > 0) {
         prof_before(1, stream);
-        kern<<<grid, C::THREADS, C::SMEM, stream>>>(mq, mk, mv, mdo, mdk, mdv, p);
+        if (launch_dependent(kern, dim3(grid), dim3(C::THREADS), C::SMEM, stream, mq, mk, mv, mdo, mdk, mdv, p) !=
+            cudaSuccess)
+            return 5;
         prof_after(1, stream);
-        if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
     if (!DQ) return launch_bwd_dq(pr, dout, lse2, delta, dq, dev, stream);
-    dim3 cg((pr.Tq + 31) / 32, pr.Hq);
-    bwd_convert_kernel<D><<<cg, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16*>(dq), pr.Tq, pr.Hq, pr.scale);
-    return cudaPeekAtLastError() == cudaSuccess ? 0 : 5;
+    const dim3 cg((pr.Tq + 31) / 32, pr.Hq);
+    if (launch_dependent(bwd_convert_kernel<D>, cg, dim3(256), 0, stream, static_cast<const float*>(dq_acc),
+                         static_cast<__nv_bfloat16*>(dq), pr.Tq, pr.Hq, pr.scale) != cudaSuccess)
+        return 5;
+    return 0;
 }
 
 // Head dim 128, deterministic: the two-items-in-flight main kernel, then the dQ pass.

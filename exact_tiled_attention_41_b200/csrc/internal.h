@@ -3,6 +3,8 @@
 #pragma once
 
 #include <cuda_runtime.h>
+
+#include <utility>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -43,6 +45,25 @@ int get_device(Device* dev);     // fills for the current device; returns FA sta
 // optional CUDA-event timing around a main-kernel launch (see fa_profile_begin)
 void prof_before(int kernel_id, cudaStream_t s);
 void prof_after(int kernel_id, cudaStream_t s);
+
+// Launch `kern` on `stream` with programmatic stream serialization: its CTAs may be scheduled before the
+// previous kernel on the stream has finished and run until their grid_dep_wait(), which returns once
+// that kernel has completed.  (With an event recorded in between, the launch is serialized as usual.)
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                             Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 int launch_fwd(const Problem& pr, void* out, float* lse, int* counter, const Device& dev, cudaStream_t stream);
 

@@ -285,6 +285,13 @@ __device__ __forceinline__ void umma_ts_lo(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic-serialization attribute may start
+// before the previous kernel on its stream has finished; grid_dep_wait() blocks until that kernel has
+// completed and its memory writes are visible (it returns at once for an ordinary launch), and
+// grid_dep_launch() lets the next such kernel start once every CTA of this grid has called it or exited.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Arrive once on `bar` when every tcgen05 operation issued so far by this thread has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
