@@ -126,6 +126,10 @@ __global__ void __launch_bounds__((kDecConsumers + 1) * 32, dec_min_blocks<D>())
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kDecStages * STAGE_BYTES);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * kDecStages);
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + kDecStages);
+    // launched with programmatic serialization: everything the previous kernel on the stream wrote (the
+    // appended cache rows, the lengths, the previous call's use of the partials) is settled after this
+    grid_dep_wait();
+    grid_dep_launch();
 
     const int chunk_id = blockIdx.x, b = blockIdx.z;
     const int hk = blockIdx.y / p.row_blocks, rb = blockIdx.y % p.row_blocks;
@@ -382,6 +386,7 @@ __global__ void __launch_bounds__((kDecConsumers + 1) * 32, dec_min_blocks<D>())
 template <int D>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const __grid_constant__ DecodeParams p,
                                                              __nv_bfloat16* out, float* lse, int B) {
+    grid_dep_wait();   // the split kernel's partials
     const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (gw >= B * p.Sq * p.Hq) return;
@@ -422,6 +427,7 @@ __global__ void __launch_bounds__(256) kv_append_kernel(const __grid_constant__ 
                                                         __nv_bfloat16* k_cache, __nv_bfloat16* v_cache,
                                                         const __nv_bfloat16* k_new, const __nv_bfloat16* v_new,
                                                         int B, int Sn) {
+    grid_dep_launch();   // the split kernel may be scheduled; it waits for this grid before reading
     const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     if (gw >= static_cast<long long>(B) * Sn * p.Hkv) return;
@@ -503,11 +509,12 @@ int kvcache_chunk(const KvCall& c, int num_sms) {
     if (c.num_splits > 0) {
         ch = (static_cast<long long>(cap) + c.num_splits - 1) / c.num_splits;
     } else {
-        // aim for ~8 splits per CTA slot (2 CTAs per SM), assuming caches half full on average, but at
-        // least 512 keys per split: shorter splits spend a large share of their time starting up
-        // (measured on B200 with 64 rows x 8 KV heads of 1-2K keys: 256-key splits 4.0 TB/s, 512-key 4.9)
-        ch = parallel * cap / (2LL * 8 * 2 * num_sms);
-        if (ch > 1024) ch = 1024;
+        // aim for about 6 waves of split CTAs (2 per SM), assuming caches half full on average, with at
+        // least 512 keys per split: shorter splits spend a large share of their time starting up (B200, 64
+        // rows x 8 KV heads of 1-2K keys: 256-key splits 4.0 TB/s, 512-key 4.9), while on long caches fewer,
+        // longer splits cut the partial-output traffic (64 rows x 8 KV heads of 1-16K keys, 1 / 4 new tokens:
+        // 16 splits of 1024 keys 6.38 / 5.54 TB/s, 8 splits 6.66 / 6.17, 6 splits 6.72 / 6.35)
+        ch = parallel * cap / (2LL * 6 * 2 * num_sms);
         if (ch < 512) ch = 512;
     }
     ch = (ch + kDecTile - 1) / kDecTile * kDecTile;
@@ -584,13 +591,14 @@ static int run_decode(const KvCall& c, int chunk, void* workspace, const Device&
     }
     dim3 grid(p.max_chunks, c.Hkv * p.row_blocks, c.B);
     prof_before(2, stream);
-    kern<<<grid, (kDecConsumers + 1) * 32, smem, stream>>>(mk, mv, p);
+    if (launch_dependent(kern, grid, dim3((kDecConsumers + 1) * 32), smem, stream, mk, mv, p) != cudaSuccess)
+        return FA_ERR_CUDA;
     prof_after(2, stream);
-    if (cudaPeekAtLastError() != cudaSuccess) return FA_ERR_CUDA;
     const long long warps = static_cast<long long>(c.B) * c.Sq * c.Hq;
-    decode_combine_kernel<D><<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(
-        p, static_cast<__nv_bfloat16*>(c.out), c.lse, c.B);
-    return cudaPeekAtLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    if (launch_dependent(decode_combine_kernel<D>, dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, stream,
+                         p, static_cast<__nv_bfloat16*>(c.out), c.lse, c.B) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return FA_OK;
 }
 
 int kvcache_launch(const KvCall& c, int chunk, void* workspace, const Device& dev, cudaStream_t stream) {

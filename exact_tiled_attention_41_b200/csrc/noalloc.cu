@@ -72,12 +72,19 @@ extern "C" int fa_fwd_kvcache_noalloc(const void* q, const void* k_cache, const 
     const int st0 = kvcache_validate(c, true);
     if (st0 != FA_OK) return st0;
 
-    // Split size: the usual choice, made coarser (auto mode only) until the partials fit the fixed array.
+    // Split size: the usual choice; in automatic mode, when its partials do not fit the fixed array, the
+    // largest smaller split count that fits (each count split exactly as num_splits = n splits it).
     const int cap = kvcache_chunk_limit(c);
     int chunk = kvcache_chunk(c, 148);
-    while (kvcache_workspace_bytes(c, chunk) > kNoAllocScratchBytes) {
-        if (num_splits > 0 || chunk >= cap) return FA_ERR_WORKSPACE;   // beyond the fixed maximum
-        chunk = chunk * 2 > cap ? (cap + 63) / 64 * 64 : chunk * 2;
+    if (kvcache_workspace_bytes(c, chunk) > kNoAllocScratchBytes) {
+        if (num_splits > 0) return FA_ERR_WORKSPACE;                   // an explicit split is not changed
+        KvCall cn = c;
+        for (int n = (cap + chunk - 1) / chunk - 1;; --n) {
+            if (n < 1) return FA_ERR_WORKSPACE;                        // one split per row does not fit either
+            cn.num_splits = n;
+            chunk = kvcache_chunk(cn, 148);
+            if (kvcache_workspace_bytes(c, chunk) <= kNoAllocScratchBytes) break;
+        }
     }
 
     Device dev;

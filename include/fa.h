@@ -284,9 +284,11 @@ FA_API int fa_merge_lse(const void* o_parts, const float* lse_parts, int num_par
  *   - All calls share the array: calls that overlap on the GPU (other streams,
  *     other host threads) race on it and must be serialised by the caller.
  *     Nothing in it needs to start at zero; each call writes what it reads.
- *   - With num_splits = 0 the split is chosen as for fa_fwd_kvcache and made
- *     coarser (doubled, at most to the whole capacity) until the partials fit;
- *     when no coarsening is needed the result is bit-identical to fa_fwd_kvcache's.  If they cannot fit (an explicit
+ *   - With num_splits = 0 the split is chosen as for fa_fwd_kvcache; when its
+ *     partials do not fit, the largest smaller split count n whose partials fit
+ *     is used, split exactly as fa_fwd_kvcache splits with num_splits = n, so the
+ *     result is bit-identical to that call's (and to the num_splits = 0 call's
+ *     when no coarsening is needed).  If they cannot fit (an explicit
  *     num_splits too large, or B * Sq * Hq * (D + 1) * 4 bytes beyond the array),
  *     the call returns FA_ERR_WORKSPACE and launches nothing.
  */

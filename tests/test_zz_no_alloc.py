@@ -59,12 +59,22 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(D):
         assert torch.equal(lse, ref_lse), f"call {call}: LSE differs from fa_fwd_kvcache"
 
 
+def _partial_bytes(B, Hkv, rows, D, cap, n):
+    # the partials of n splits: the split length is ceil(cap / n) rounded up to 64 keys
+    chunk = -(-(-(-cap // n)) // 64) * 64
+    chunks = -(-cap // chunk)
+    r = B * Hkv * chunks * rows
+    return (r * D * 4 + 255) // 256 * 256 + r * 4
+
+
 def test_noalloc_coarsens_the_split_until_the_partials_fit():
-    # 64 rows x 8 KV heads x 16 query rows (4 heads per KV head x 4 causal tokens), capacity 4096: the
-    # usual 512-key split needs 8 partials per (row, KV head) -- 33.8 MB; 1024 keys still need 16.9 MB
-    # > 16 MiB, so the call runs two splits of 2048 keys (8.5 MB), the split fa_fwd_kvcache takes with
-    # num_splits = 2
+    # 64 rows x 8 KV heads x 16 query rows (4 heads per KV head x 4 causal tokens), capacity 4096: four
+    # splits of 1024 keys need 16.9 MB of partials > 16 MiB, three splits of 1408 keys 12.7 MB, so the call
+    # runs the split fa_fwd_kvcache takes with num_splits = 3 (the automatic split has more than three)
     B, Hq, Hkv, D, cap, Sq = 64, 32, 8, 128, 4096, 4
+    limit = abi.fa_fwd_kvcache_noalloc_scratch_bytes()
+    n_fit = max(n for n in range(1, 9) if _partial_bytes(B, Hkv, Sq * Hq // Hkv, D, cap, n) <= limit)
+    assert n_fit == 3
     g = torch.Generator("cpu").manual_seed(40)
     lengths = torch.randint(Sq, 200, (B,), generator=g).tolist()
     lengths[3], lengths[17], lengths[40] = cap, 2049, 2048
@@ -72,7 +82,7 @@ def test_noalloc_coarsens_the_split_until_the_partials_fit():
     t = {n: x.cuda() for n, x in w.tensors.items()}
     for _ in range(2):
         out, lse = _noalloc(t, B, Hq, Hkv, cap, D, w.scale, Sq, 1)
-        ref_out, ref_lse = _reference(t, B, Hq, Hkv, cap, D, w.scale, 2, Sq, 1)
+        ref_out, ref_lse = _reference(t, B, Hq, Hkv, cap, D, w.scale, n_fit, Sq, 1)
         assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
     # and against the fp64 oracle on the rows' valid keys (bottom-right causal tokens)
     L = max(lengths)
