@@ -10,7 +10,8 @@
 // (128 x 256 each), a ring of five 16 KB slots for the Q and dO tiles (see Cfg)
 // and dS^T fit shared memory.
 //   tensor memory: dV half [0,128) | dK half [128,256) | S^T [256,320) |
-//                  dP^T [320,384) | dQ^T half [384,448)
+//                  dP^T [320,384) | dQ^T half [384,448); after the gradient step each
+//                  32-query half's packed P^T and dS^T sit in that half's S^T columns
 //   dQ^T = K_half^T dS^T has the head dimension on the 128 lanes, so the dQ
 //   warpgroup's atomics cover 32 consecutive head-dim floats per warp and the
 //   accumulator is laid out [Hq][Tq][256].
@@ -116,13 +117,16 @@ struct Cfg {
                               OFF_STAT = OFF_DS + 128 * 128,            // [2][-LSE2 x 64 | -Delta x 64]
                               OFF_BAR = OFF_STAT + 2 * 128 * 4;
     // kv_full, kv_empty | slot_full[NSLOT] | slot_empty[NSLOT] | stat_full[2] | stat_empty[2] |
-    // s_full, p_full, dq_full, dq_empty, dkv_full, dk_done, dv_done | unit feed
+    // s_full, p_full, dq_full, dq_empty, dkv_full, (unused), dv_done | unit feed
     static constexpr int BAR_SLOT_FULL = 2, BAR_SLOT_EMPTY = 2 + NSLOT, BAR_STAT_FULL = 2 + 2 * NSLOT,
                          BAR_STAT_EMPTY = BAR_STAT_FULL + 2, BAR_S_FULL = BAR_STAT_EMPTY + 2, BAR_FEED = BAR_S_FULL + 7;
     static constexpr int NUM_BARS = BAR_FEED + 2 * kFeedSlots;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
     static_assert(SMEM <= 232448, "shared memory per block");
     static constexpr uint32_t COL_DV = 0, COL_DK = 128, COL_S = 256, COL_DP = 320, COL_DQ = 384;
+    // packed P^T of queries [16 kk, 16 kk + 16) (8 columns of bf16 pairs): compute warpgroup kk / 2 wrote
+    // them into the first 16 of the 32 S^T columns it read; dS^T of the same queries sits 16 columns later
+    static constexpr uint32_t COL_PK(int kk) { return COL_S + 32 * (kk >> 1) + 8 * (kk & 1); }
     // 16 warps: 0-7 two compute warpgroups (query columns 0-31 / 32-63), 8-11 dQ warpgroup, 12 producer,
     // 13 and 14 the two MMA issuers, 15 idle.  Registers: launch at 128 per thread (512 x 128 = 65536); the
     // producer / issuer warpgroup gives 40 per thread to the dQ warpgroup.  The host checks the launch count.
@@ -132,9 +136,9 @@ struct Cfg {
 
 // One issuing thread takes about 54 cycles per 16-deep MMA, more than the tensor core needs for the 128 x 64
 // products here, so two threads issue: A takes S^T, dQ^T and dK (the Q pairs are its operands), B takes dP^T
-// and dV (the dO pairs).  Each releases the ring slots of its own pairs.  S^T of a tile overwrites the P^T
-// that B's dV of the previous tile reads, and dP^T overwrites the dS^T that A's dK reads, so each issuer
-// waits for the other's previous product there (dv_done, dk_done).
+// and dV (the dO pairs).  Each releases the ring slots of its own pairs.  S^T of a tile overwrites the
+// packed P^T and dS^T of the previous tile (in the S^T columns), read by B's dV and A's own dK, so A waits
+// for B's previous dV there (dv_done).
 template <bool DQ>
 __global__ void __launch_bounds__(512, 1)
     bwd256_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -155,7 +159,7 @@ __global__ void __launch_bounds__(512, 1)
     auto stat_full = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_FULL + s); };
     auto stat_empty = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_EMPTY + s); };
     const uint32_t s_full = b0 + 8u * C::BAR_S_FULL, p_full = s_full + 8, dq_full = s_full + 16,
-                   dq_empty = s_full + 24, dkv_full = s_full + 32, dk_done = s_full + 40, dv_done = s_full + 48;
+                   dq_empty = s_full + 24, dkv_full = s_full + 32, dv_done = s_full + 48;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PRODUCER = 12, MMA_A = 13, MMA_B = 14;
 
@@ -179,7 +183,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bars + C::BAR_S_FULL + 2, 1);                      // dq_full
         mbar_init(bars + C::BAR_S_FULL + 3, 128);                    // dq_empty
         mbar_init(bars + C::BAR_S_FULL + 4, 2);                      // dkv_full: last dK (A) and dV (B)
-        mbar_init(bars + C::BAR_S_FULL + 5, 1);                      // dk_done
+        mbar_init(bars + C::BAR_S_FULL + 5, 1);                      // (unused)
         mbar_init(bars + C::BAR_S_FULL + 6, 1);                      // dv_done
         for (int s = 0; s < kFeedSlots; ++s) {
             mbar_init(bars + C::BAR_FEED + s, 1);                              // unit published
@@ -298,8 +302,7 @@ __global__ void __launch_bounds__(512, 1)
                 const uint32_t k_other = isA ? 0u : 1u, k_own = isA ? 2u : 3u;
                 const uint32_t col_s = isA ? C::COL_S : C::COL_DP;                     // S^T or dP^T
                 const uint32_t col_g = isA ? C::COL_DK : C::COL_DV;                    // dK or dV
-                const uint32_t col_a = isA ? C::COL_DP : C::COL_S;                     // dS^T or P^T (A operand)
-                const uint32_t done_mine = isA ? dk_done : dv_done, done_other = isA ? dv_done : dk_done;
+                const uint32_t a_off = isA ? 16u : 0u;                                 // packed dS^T or P^T
                 uint32_t unit_it = 0, q_it = 0;
                 bool ok = true;
                 for (uint32_t fi = 0; ok; ++fi) {
@@ -319,7 +322,8 @@ __global__ void __launch_bounds__(512, 1)
                         const uint32_t po = dRK + slo * PAIR16, ph = dRK + sho * PAIR16, phn = dRN + sho * PAIR16;
                         if (!mbar_wait(slot_full(slo), ((px + k_other) / C::NSLOT) & 1, w)) { ok = false; break; }
                         // the other issuer's product of the previous tile has read what this one overwrites
-                        if (q_it > 0 && !mbar_wait(done_other, (q_it - 1) & 1, w)) { ok = false; break; }
+                        // S^T overwrites the packed P^T / dS^T of the previous tile, read by B's dV (and A's dK)
+                        if (isA && q_it > 0 && !mbar_wait(dv_done, (q_it - 1) & 1, w)) { ok = false; break; }
                         if (isA && !mbar_wait(slot_full(sho), ((px + k_own) / C::NSLOT) & 1, w)) { ok = false; break; }
                         tc_fence_after();
                         // S^T = K Q^T (A) or dP^T = V dO^T (B) over the head dim, the other half's chunks first
@@ -355,9 +359,10 @@ __global__ void __launch_bounds__(512, 1)
                         const uint32_t first = it > 0 ? 1u : 0u;
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
-                            umma_ts_lo(tmem + col_g, tmem + col_a + kk * 8, phn + kk * ROWS16, id_g, kk > 0 ? 1u : first);
+                            umma_ts_lo(tmem + col_g, tmem + C::COL_PK(kk) + a_off, phn + kk * ROWS16, id_g,
+                                       kk > 0 ? 1u : first);
                         umma_commit(slot_empty(sho));             // the own-half pair: last read here
-                        umma_commit(done_mine);
+                        if (!isA) umma_commit(dv_done);
                     }
                     if (!ok) break;
                     umma_commit(dkv_full);
@@ -502,8 +507,10 @@ __global__ void __launch_bounds__(512, 1)
                     pp[e / 2] = pack_bf16x2(pr.x, pr.y);
                     dd[e / 2] = pack_bf16x2(ds.x, ds.y);
                 }
-                tmem_st16(tmem + lb + C::COL_S + 16 * gq, pp);
-                tmem_st16(tmem + lb + C::COL_DP + 16 * gq, dd);
+                // P^T and dS^T of this warpgroup's 32 queries go back into the 32 S^T columns it has just
+                // read (16 each), so neither warpgroup writes columns the other still reads
+                tmem_st16(tmem + lb + C::COL_S + 32 * gq, pp);
+                tmem_st16(tmem + lb + C::COL_S + 32 * gq + 16, dd);
                 uint8_t* ds_row = smem + C::OFF_DS + r * 128;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
