@@ -117,9 +117,9 @@ struct Cfg {
                               OFF_STAT = OFF_DS + 128 * 128,            // [2][-LSE2 x 64 | -Delta x 64]
                               OFF_BAR = OFF_STAT + 2 * 128 * 4;
     // kv_full, kv_empty | slot_full[NSLOT] | slot_empty[NSLOT] | stat_full[2] | stat_empty[2] |
-    // s_full, p_full, dq_full, dq_empty, dkv_full, (unused), dv_done | unit feed
+    // s_full, p_full, dq_full, dq_empty, dkv_full, dv_done | unit feed
     static constexpr int BAR_SLOT_FULL = 2, BAR_SLOT_EMPTY = 2 + NSLOT, BAR_STAT_FULL = 2 + 2 * NSLOT,
-                         BAR_STAT_EMPTY = BAR_STAT_FULL + 2, BAR_S_FULL = BAR_STAT_EMPTY + 2, BAR_FEED = BAR_S_FULL + 7;
+                         BAR_STAT_EMPTY = BAR_STAT_FULL + 2, BAR_S_FULL = BAR_STAT_EMPTY + 2, BAR_FEED = BAR_S_FULL + 6;
     static constexpr int NUM_BARS = BAR_FEED + 2 * kFeedSlots;
     static constexpr size_t SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 4 * kFeedSlots;
     static_assert(SMEM <= 232448, "shared memory per block");
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(512, 1)
     auto stat_full = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_FULL + s); };
     auto stat_empty = [&](uint32_t s) { return b0 + 8u * (C::BAR_STAT_EMPTY + s); };
     const uint32_t s_full = b0 + 8u * C::BAR_S_FULL, p_full = s_full + 8, dq_full = s_full + 16,
-                   dq_empty = s_full + 24, dkv_full = s_full + 32, dv_done = s_full + 48;
+                   dq_empty = s_full + 24, dkv_full = s_full + 32, dv_done = s_full + 40;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     constexpr int PRODUCER = 12, MMA_A = 13, MMA_B = 14;
 
@@ -183,8 +183,7 @@ __global__ void __launch_bounds__(512, 1)
         mbar_init(bars + C::BAR_S_FULL + 2, 1);                      // dq_full
         mbar_init(bars + C::BAR_S_FULL + 3, 128);                    // dq_empty
         mbar_init(bars + C::BAR_S_FULL + 4, 2);                      // dkv_full: last dK (A) and dV (B)
-        mbar_init(bars + C::BAR_S_FULL + 5, 1);                      // (unused)
-        mbar_init(bars + C::BAR_S_FULL + 6, 1);                      // dv_done
+        mbar_init(bars + C::BAR_S_FULL + 5, 1);                      // dv_done
         for (int s = 0; s < kFeedSlots; ++s) {
             mbar_init(bars + C::BAR_FEED + s, 1);                              // unit published
             mbar_init(bars + C::BAR_FEED + kFeedSlots + s, DQ ? 14 : 10);      // read by the issuers, compute (, dQ) warps
