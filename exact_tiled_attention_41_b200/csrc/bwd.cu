@@ -10,7 +10,8 @@
 //
 // Three launches:
 //   1. preprocess: Delta = rowsum(dO * O) in fp32, LSE2 = LSE * log2(e) (+inf for
-//      rows with no key, so their P is exactly 0), and a zeroed fp32 dQ accumulator.
+//      rows with no key, so their P is exactly 0), and a zeroed fp32 dQ accumulator
+//      (kept in L2 up to the convert when it is small enough: kBwdL2KeepBytes).
 //   2. main kernel, one persistent CTA per SM, KV-tile stationary: a work unit
 //      is (sequence, KV head, 128-key tile); it loops over the 128-row query
 //      tiles of every query head that reads the KV head (so dK and dV of GQA
@@ -36,7 +37,7 @@
 //                    (tensor-memory A), while warpgroup 1 still works; then
 //                    dQ = dS K, all D columns in one product, into dP^T's columns,
 //                    so the dQ read-out overlaps the dV, dK products over queries 64-127
-//   3. convert: dQ = bf16(scale * dQacc).
+//   3. convert: dQ = bf16(scale * dQacc); the dead accumulator's L2 lines are discarded.
 // The deterministic backward runs the main kernel with DQ = false (no dQ product,
 // no reduce-adds, warps 8-11 idle) and computes dq in the query-tile-stationary
 // pass of bwd_dq.cu instead of steps 2's dQ and 3.
@@ -57,6 +58,11 @@ namespace fa {
 // in kBwdFmaExpEvery, 0 = none.
 constexpr int kBwdFmaExpEvery = FA_BWD_FMA_EXP_EVERY;
 
+// A dQ accumulator of at most this many bytes (about half of the 126 MB L2) is kept in L2 from the
+// preprocess to the convert with the evict_last policy (the dense prefill workload's is 64 MiB: +1.7 % on
+// the whole backward; larger ones would push out the Q and dO tiles that the key tiles share).
+constexpr size_t kBwdL2KeepBytes = size_t(64) << 20;
+
 struct BwdParams {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
@@ -71,6 +77,7 @@ struct BwdParams {
     int wl, wr;             // window sides, -1 = unbounded; a causal mask is wr = 0
     int chunk;              // (sequence, KV head) groups per chunk of the unit list
     int* counter;           // unit counter of the dynamic schedule (zeroed by the preprocess kernel)
+    int l2_keep;            // 1: reduce-adds into dQacc with the L2 evict_last policy
     unsigned long long timeout_ns;
     int* status;
 };
@@ -395,6 +402,7 @@ __global__ void __launch_bounds__(512, 1)
         const int wq = warp - 8;
         const int r = wq * 32 + lane;
         const uint32_t lb = tmem_lane_base(wq);
+        const uint64_t acc_pol = p.l2_keep ? l2_policy_last() : l2_policy_normal();
         uint32_t g_it = 0;
         bool ok = true;
         for (uint32_t fi = 0; ok; ++fi) {
@@ -427,9 +435,11 @@ __global__ void __launch_bounds__(512, 1)
                     for (int cc = 0; cc < D / 32; ++cc)
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            atomicAdd(acc + static_cast<size_t>(cc * 8 + e) * p.Tq,
-                                      make_float4(__uint_as_float(ra[cc][4 * e]), __uint_as_float(ra[cc][4 * e + 1]),
-                                                  __uint_as_float(ra[cc][4 * e + 2]), __uint_as_float(ra[cc][4 * e + 3])));
+                            red_add_f32x4_hint(acc + static_cast<size_t>(cc * 8 + e) * p.Tq,
+                                               make_float4(__uint_as_float(ra[cc][4 * e]), __uint_as_float(ra[cc][4 * e + 1]),
+                                                           __uint_as_float(ra[cc][4 * e + 2]),
+                                                           __uint_as_float(ra[cc][4 * e + 3])),
+                                               acc_pol);
                 }
             }
         }
@@ -1000,24 +1010,28 @@ __global__ void __launch_bounds__(384, 1)
 // ---------------------------------------------------------------------------- preprocess
 // One warp per (query token, head): Delta = sum_d dO * O (fp32), LSE2 = LSE * log2(e)
 // (+inf where LSE = -inf).  Also zeroes the dQ accumulator (grid-stride) unless dq_acc is NULL, and
-// the main kernel's unit counter unless counter is NULL.
+// the main kernel's unit counter unless counter is NULL.  With l2_keep the zeroed accumulator is
+// written with the L2 evict_last policy and O, dO are read with evict_first, so that the accumulator
+// stays in L2 for the main kernel's reduce-adds and the convert.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, const __nv_bfloat16* dout,
                                                       const float* lse, float* lse2, float* delta, float* dq_acc,
                                                       int* counter, int Tq, int Hq, int Sq, long long lse_sB,
-                                                      long long lse_sH, int lse_sT) {
+                                                      long long lse_sH, int lse_sT, int l2_keep) {
     const long long gw = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int lane = threadIdx.x & 31;
     // the main kernel may start its prologue now; it waits for this grid before reading anything written here
     if (threadIdx.x == 0) grid_dep_launch();
     if (counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *counter = 0;
     const long long rows = static_cast<long long>(Tq) * Hq;
+    const uint64_t pol_in = l2_keep ? l2_policy_first() : l2_policy_normal();
     if (dq_acc != nullptr) {
+        const uint64_t pol_z = l2_keep ? l2_policy_last() : l2_policy_normal();
         const long long n4 = rows * D / 4;
         float4* z = reinterpret_cast<float4*>(dq_acc);
         for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
              i += static_cast<long long>(gridDim.x) * blockDim.x)
-            z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+            st_f32x4_hint(z + i, make_float4(0.f, 0.f, 0.f, 0.f), pol_z);
     }
     // D/8 lanes per row, 16 bytes of O and of dO per lane; 32/(D/8) rows per warp per pass
     constexpr int LPR = D / 8, RPW = 32 / LPR;
@@ -1027,8 +1041,8 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
         const long long row = row0 + sub;
         float s = 0.f;
         if (row < rows) {
-            const uint4 a = *reinterpret_cast<const uint4*>(out + row * D + sl * 8);
-            const uint4 b = *reinterpret_cast<const uint4*>(dout + row * D + sl * 8);
+            const uint4 a = ld_u32x4_hint(out + row * D + sl * 8, pol_in);
+            const uint4 b = ld_u32x4_hint(dout + row * D + sl * 8, pol_in);
             const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -1062,7 +1076,9 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
 // of 32 consecutive tokens are read (512 bytes per warp), staged in shared memory with one float4 of padding
 // per token row (each group of 8 lanes then writes 8 different bank groups), and leave as whole D-value rows
 // (D / 8 lanes x 16 bytes per token).  Launched after the main kernel with programmatic serialization: the
-// wait below covers the main kernel's last reduce-adds.
+// wait below covers the main kernel's last reduce-adds.  The accumulator is dead once read: the 128-byte
+// L2 lines that lie wholly inside this block's token range are dropped without being written back (a line
+// shared with a neighbouring block is left alone), which saves its write-back to HBM.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_convert_kernel(const float* dq_acc, __nv_bfloat16* dq, int Tq, int Hq,
                                                           float scale) {
@@ -1077,6 +1093,15 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(const float* dq_acc, _
         if (t0 + tt < Tq) tile[tt * W4 + d4] = __ldcs(src + static_cast<size_t>(d4) * Tq + tt);
     }
     __syncthreads();
+    if (threadIdx.x < (D / 4) * 4) {
+        // row d4 of this head: bytes [16 (rowbase + t0), 16 (rowbase + t1)) of the accumulator, whose base
+        // is 256-byte aligned; line k of the whole lines inside that range
+        const int d4 = threadIdx.x >> 2, k = threadIdx.x & 3;
+        const long long rowbase = (static_cast<long long>(h) * (D / 4) + d4) * Tq;
+        const long long b0 = (rowbase + t0) * 16, b1 = (rowbase + min(t0 + 32, Tq)) * 16;
+        const long long line = ((b0 + 127) & ~127LL) + 128LL * k;
+        if (line + 128 <= b1) l2_discard_line(reinterpret_cast<const char*>(dq_acc) + line);
+    }
     constexpr int LPR = D / 8;                     // lanes per token row, 8 values (16 bytes) each
     for (int i = threadIdx.x; i < 32 * LPR; i += blockDim.x) {
         const int tt = i / LPR, c8 = i % LPR;
@@ -1127,6 +1152,8 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     float* dq_acc = static_cast<float*>(workspace);
     float* lse2 = reinterpret_cast<float*>(static_cast<char*>(workspace) + up(static_cast<size_t>(pr.Tq) * pr.Hq * D * 4));
     float* delta = reinterpret_cast<float*>(reinterpret_cast<char*>(lse2) + up(static_cast<size_t>(pr.Tq) * pr.Hq * 4));
+    const size_t acc_bytes = static_cast<size_t>(pr.Tq) * pr.Hq * D * 4;
+    const int l2_keep = (DQ && acc_bytes <= kBwdL2KeepBytes) ? 1 : 0;
 
     {
         const long long rows = static_cast<long long>(pr.Tq) * pr.Hq;
@@ -1136,7 +1163,7 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
         bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
             DQ ? dq_acc : nullptr, bwd_unit_counter(workspace, pr.Tq, pr.Hq, D), pr.Tq, pr.Hq, pr.Sq, pr.lse_sB,
-            pr.lse_sH, pr.lse_sT);
+            pr.lse_sH, pr.lse_sT, l2_keep);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
 
@@ -1175,6 +1202,7 @@ static int run_bwd(const Problem& pr, const void* out, const void* dout, const f
     p.wl = pr.wl;
     p.wr = pr.wr;
     p.chunk = bwd_chunk_groups(pr.num_seqs * pr.Hkv, p.n_blocks, p.group, pr.Sq, D, dev.num_sms);
+    p.l2_keep = l2_keep;
     p.counter = bwd_unit_counter(workspace, pr.Tq, pr.Hq, D);
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
@@ -1222,7 +1250,7 @@ static int run_bwd_pp(const Problem& pr, const void* out, const void* dout, cons
         if (blocks > cap) blocks = cap;
         bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
             static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
-            nullptr, nullptr, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT);
+            nullptr, nullptr, pr.Tq, pr.Hq, pr.Sq, pr.lse_sB, pr.lse_sH, pr.lse_sT, 0);
         if (cudaPeekAtLastError() != cudaSuccess) return 5;
     }
     alignas(64) CUtensorMap mq, mk, mv, mdo;
@@ -1257,6 +1285,7 @@ static int run_bwd_pp(const Problem& pr, const void* out, const void* dout, cons
     p.wl = pr.wl;
     p.wr = pr.wr;
     p.chunk = pr.num_seqs * pr.Hkv;   // the static heaviest-first order over all groups
+    p.l2_keep = 0;
     p.counter = nullptr;
     p.timeout_ns = dev.timeout_ns;
     p.status = dev.status;
@@ -1297,7 +1326,7 @@ static int run_bwd256(const Problem& pr, const void* out, const void* dout, cons
     bwd_pre_kernel<D><<<static_cast<int>(blocks), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(out), static_cast<const __nv_bfloat16*>(dout), lse, lse2, delta,
         det ? nullptr : dq_acc, bwd_unit_counter(workspace, pr.Tq, pr.Hq, D), pr.Tq, pr.Hq, pr.Sq, pr.lse_sB,
-        pr.lse_sH, pr.lse_sT);
+        pr.lse_sH, pr.lse_sT, 0);
     if (cudaPeekAtLastError() != cudaSuccess) return 5;
     const int st = launch_bwd256_main(pr, dout, lse2, delta, dq_acc, dq, dk, dv, !det, dev, stream);
     if (st != 0 || !det) return st;

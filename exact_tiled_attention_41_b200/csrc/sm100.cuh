@@ -376,6 +376,48 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
     return make_float2(__uint_as_float(bx), __uint_as_float(by));
 }
 
+// ------------------------------------------------------------------ L2 eviction priority
+// Cache policies for the .L2::cache_hint forms of loads, stores and reductions: lines brought in or
+// written with evict_last are replaced after the others, evict_first before them, evict_normal as
+// without a hint.  The hint changes no value, only which lines L2 keeps.
+__device__ __forceinline__ uint64_t l2_policy_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_normal() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void red_add_f32x4_hint(float4* addr, float4 v, uint64_t pol) {
+    asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr), "f"(v.x),
+                 "f"(v.y), "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ void st_f32x4_hint(float4* addr, float4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(addr), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 ld_u32x4_hint(const void* addr, uint64_t pol) {
+    uint4 v;
+    asm volatile("ld.global.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(addr), "l"(pol));
+    return v;
+}
+// Drop one 128-byte L2 line without writing it back: its contents become undefined.  addr must be
+// 128-byte aligned, and no other thread may still read the line.
+__device__ __forceinline__ void l2_discard_line(const void* addr) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(addr) : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
