@@ -63,6 +63,11 @@ constexpr int kBwdFmaExpEvery = FA_BWD_FMA_EXP_EVERY;
 // the whole backward; larger ones would push out the Q and dO tiles that the key tiles share).
 constexpr size_t kBwdL2KeepBytes = size_t(64) << 20;
 
+#ifndef FA_BWD_PRE_PASSES
+#define FA_BWD_PRE_PASSES 1
+#endif
+constexpr int kPrePasses = FA_BWD_PRE_PASSES;
+
 struct BwdParams {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
@@ -1033,17 +1038,45 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
              i += static_cast<long long>(gridDim.x) * blockDim.x)
             st_f32x4_hint(z + i, make_float4(0.f, 0.f, 0.f, 0.f), pol_z);
     }
-    // D/8 lanes per row, 16 bytes of O and of dO per lane; 32/(D/8) rows per warp per pass
-    constexpr int LPR = D / 8, RPW = 32 / LPR;
-    const int sub = lane / LPR, sl = lane % LPR;
+    // D/8 lanes per row, 16 bytes of O and of dO per lane; 32/(D/8) rows per warp per pass.  A row's LSE is
+    // loaded together with its O and dO, so that a pass waits for one round trip to memory rather than two,
+    // and each iteration takes kPrePasses passes, whose loads are all in flight at once.
+    constexpr int LPR = D / 8, RPW = 32 / LPR, NP = kPrePasses;
     const long long nwarps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-    for (long long row0 = gw * RPW; row0 < rows; row0 += nwarps * RPW) {
-        const long long row = row0 + sub;
-        float s = 0.f;
-        if (row < rows) {
-            const uint4 a = ld_u32x4_hint(out + row * D + sl * 8, pol_in);
-            const uint4 b = ld_u32x4_hint(dout + row * D + sl * 8, pol_in);
-            const uint32_t av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+    const int sub = lane / LPR, sl = lane % LPR;
+    const long long stride = nwarps * RPW;
+    for (long long row0 = gw * RPW; row0 < rows; row0 += NP * stride) {
+        uint4 a[NP], b[NP];
+        float l[NP];
+        size_t wi[NP];
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const long long row = row0 + k * stride + sub;
+            a[k] = make_uint4(0, 0, 0, 0);
+            b[k] = a[k];
+            l[k] = 0.f;
+            wi[k] = 0;
+            if (row < rows) {
+                a[k] = ld_u32x4_hint(out + row * D + sl * 8, pol_in);
+                b[k] = ld_u32x4_hint(dout + row * D + sl * 8, pol_in);
+                const int tok = static_cast<int>(row / Hq), h = static_cast<int>(row % Hq);
+                if (sl == 0) {
+                    long long li;
+                    if (lse_sT) {
+                        li = h * lse_sH + tok;
+                    } else {
+                        const int bb = tok / Sq, i = tok - bb * Sq;
+                        li = bb * lse_sB + h * lse_sH + i;
+                    }
+                    l[k] = lse[li];
+                }
+                wi[k] = static_cast<size_t>(h) * Tq + tok;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < NP; ++k) {
+            const uint32_t av[4] = {a[k].x, a[k].y, a[k].z, a[k].w}, bv[4] = {b[k].x, b[k].y, b[k].z, b[k].w};
+            float s = 0.f;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 fa = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&av[e]));
@@ -1051,22 +1084,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* out, 
                 s = fmaf(fa.x, fb.x, s);
                 s = fmaf(fa.y, fb.y, s);
             }
-        }
 #pragma unroll
-        for (int x = LPR / 2; x > 0; x >>= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
-        if (sl == 0 && row < rows) {
-            const int tok = static_cast<int>(row / Hq), h = static_cast<int>(row % Hq);
-            long long li;
-            if (lse_sT) {
-                li = h * lse_sH + tok;
-            } else {
-                const int bb = tok / Sq, i = tok - bb * Sq;
-                li = bb * lse_sB + h * lse_sH + i;
+            for (int x = LPR / 2; x > 0; x >>= 1) s += __shfl_xor_sync(0xffffffffu, s, x);
+            if (sl == 0 && row0 + k * stride + sub < rows) {
+                lse2[wi[k]] = (l[k] == -INFINITY) ? INFINITY : l[k] * 1.4426950408889634f;
+                delta[wi[k]] = s;
             }
-            const float l = lse[li];
-            const size_t wi = static_cast<size_t>(h) * Tq + tok;
-            lse2[wi] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
-            delta[wi] = s;
         }
     }
 }
