@@ -35,6 +35,10 @@
  *   (workspace, workspace_bytes); the matching *_workspace_size() returns the
  *   bytes required (0 = none; workspace may then be NULL).  Workspace must be
  *   256-byte aligned and is not preserved between calls.
+ * - Per-device state (the status word's address, the SM count, the kernels'
+ *   shared-memory attributes) is looked up on the first call on a device and
+ *   kept for the life of the process: a cudaDeviceReset of that device after
+ *   the first call is not supported.
  *
  * Errors: every entry point returns an fa_status.  Arguments are validated
  * before anything is enqueued; a non-zero status means nothing was launched,
